@@ -1,0 +1,482 @@
+"""Benchmark of the shared-index top-k sparse KV attention hot path on B200.
+
+One bench step = one denoising block of the workload, for L independent layer
+copies (distinct K/V caches, queries and outputs, so every step streams from
+HBM rather than L2):
+  * selection of the NEXT block (dsa_select, all L layers) on a second stream,
+  * overlapped with the T-1 sparse steps of the CURRENT block
+    (dsa_sparse_attn x (T-1) x L) on the main stream, which reuse the indices
+    selected one step earlier (ping-pong index buffers).
+The step is captured once into CUDA graphs and replayed.  `value` is algorithmic
+HBM bytes (selected K/V + block Q/O per sparse step; prefix K/V + Q/O per
+selection) over device time, summed over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU runs are independent replicas (the path has no exchange step);
+torch.distributed/NCCL is used only for the barrier and the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_27_b200 import workloads as W  # noqa: E402
+
+METRIC = "sparse block-step µs & HBM GB/s (% roofline) at 128K, k=1024; select-pass ms"
+WORKLOAD_TEXT = {
+    "128k": "128k: 1 seq, prefix N=131072, block B=32, Hq=32, Hkv=8 (GQA 4), d=128, page=16, "
+            "top-k 1024 tokens (64 pages), 32 steps/block, bf16 N(0,1) with 0.5% needle pages; "
+            "selection of block n+1 on a second stream overlapped with block n's sparse steps",
+    "8k": "8k: 1 seq, N=8192, B=32, Hq=32, Hkv=8, d=128, page=16, top-k 512 tokens, 32 steps",
+    "32k": "32k: 1 seq, N=32768, B=32, Hq=28, Hkv=4, d=128, page=64, top-k 1024 tokens, 32 steps",
+    "batched": "batched: 8 seqs, N~U[16K,64K], B=32, Hq=32, Hkv=8, d=128, page=16, "
+               "top-k in {512,1024,2048}, 32 steps, random page table",
+}
+
+
+# ------------------------------------------------------------------ bytes/flops
+def sparse_bytes(w) -> int:
+    """Selected K/V + block Q/O bytes of one sparse step (per layer)."""
+    sel = sum(min(int(w.topk[s]), w.n_pages(s) * w.P) for s in range(w.S)) * w.Hkv * w.d * 2 * 2
+    qo = 2 * w.S * w.B * w.Hq * w.d * 2
+    return sel + qo
+
+
+def select_bytes(w) -> int:
+    """Prefix K/V + block Q/O bytes of one selection pass (per layer)."""
+    kv = sum(int(w.n_ctx[s]) for s in range(w.S)) * w.Hkv * w.d * 2 * 2
+    return kv + 2 * w.S * w.B * w.Hq * w.d * 2
+
+
+def sparse_flops(w) -> int:
+    keys = sum(min(int(w.topk[s]), w.n_pages(s) * w.P) + w.B for s in range(w.S)) / w.S
+    return int(4 * w.S * w.B * w.Hq * keys * w.d)
+
+
+def select_flops(w) -> int:
+    return int(4 * w.B * w.Hq * w.d * sum(int(w.n_ctx[s]) for s in range(w.S)))
+
+
+# ---------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_attention_27_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(f"{kernel}@{workload}")
+    if not rec or rec.get("source_sha") != kernel_source_sha():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in self.rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in self.rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif n_gpus > 1:
+        raise SystemExit("--gpus N > 1 must be launched with torch.distributed.run")
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- CPU baseline
+def oracle_block(w, steps):
+    """The fp64 oracle on one block of one layer: selection + `steps` sparse steps."""
+    import oracle
+    pt = None if w.page_table is None else w.page_table.numpy()
+    t0 = time.perf_counter()
+    r = oracle.select(W.bits(w.q1), W.bits(w.k_cache), W.bits(w.v_cache), w.n_ctx.numpy(),
+                      w.topk.numpy(), page_table=pt, max_pages=w.max_pages)
+    for t in range(2, 2 + steps):
+        q, bk, bv = w.step_inputs(t)
+        oracle.sparse(W.bits(q), W.bits(w.k_cache), W.bits(w.v_cache), w.n_ctx.numpy(), r.idx,
+                      r.cnt, W.bits(bk), W.bits(bv), page_table=pt, max_pages=w.max_pages)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w):
+    import oracle
+    steps = w.T - 1
+    secs = oracle_block(w, steps)
+    nbytes = select_bytes(w) + steps * sparse_bytes(w)
+    return {"value": round(nbytes / secs / 1e9, 6), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"one block of one layer of the {w.name} workload: the selection pass "
+                      f"plus {steps} sparse steps ({nbytes} algorithmic bytes) in {secs:.2f} s"}
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the fp64 oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+    w = W.make(args.workload, 0)
+    steps = w.T - 1
+    nbytes = select_bytes(w) + steps * sparse_bytes(w)
+    for _ in range(args.warmup):
+        oracle_block(w, steps)
+    secs = [oracle_block(w, steps) for _ in range(args.steps)]
+    total = sum(secs)
+    value = nbytes * args.steps / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload),
+                   "unit_of_work": "one block of one layer (selection + T-1 sparse steps)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"one block of one layer of the {args.workload} workload per "
+                                   f"step ({nbytes} algorithmic bytes)"},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU bench
+class Bench:
+    def __init__(self, w, layers: int, dsa):
+        self.w, self.L, self.dsa = w, layers, dsa
+        dev = torch.device("cuda")
+        T, S = w.T, w.S
+        self.main = torch.cuda.current_stream()   # a non-default stream set by run_ours
+        self.side = torch.cuda.Stream()
+        # L independent layer copies of the KV cache
+        self.k = torch.empty((layers, *w.k_cache.shape), dtype=torch.bfloat16, device=dev)
+        self.v = torch.empty_like(self.k)
+        kb, vb = w.k_cache.to(dev), w.v_cache.to(dev)
+        self.k.copy_(kb.unsqueeze(0).expand_as(self.k))
+        self.v.copy_(vb.unsqueeze(0).expand_as(self.v))
+        del kb, vb
+        # per-step inputs (step 1 = selection queries), one copy per layer
+        steps = [w.step_inputs(t) for t in range(1, T + 1)]
+        self.host_q = torch.stack([s[0] for s in steps]).pin_memory()     # [T, S, B, Hq, d]
+        self.host_bk = torch.stack([s[1] for s in steps]).pin_memory()    # [T, S, B, Hkv, d]
+        self.host_bv = torch.stack([s[2] for s in steps]).pin_memory()
+        self.q = self.host_q.to(dev).unsqueeze(0).repeat(layers, 1, 1, 1, 1, 1).contiguous()
+        self.bk = self.host_bk.to(dev).unsqueeze(0).repeat(layers, 1, 1, 1, 1, 1).contiguous()
+        self.bv = self.host_bv.to(dev).unsqueeze(0).repeat(layers, 1, 1, 1, 1, 1).contiguous()
+        self.n_ctx = w.n_ctx.to(dev)
+        self.topk = w.topk.to(dev)
+        self.page_table = None if w.page_table is None else w.page_table.to(dev)
+        self.dims = dsa.dims_for(self.q[0, 0], self.k[0], w.max_pages, w.kmax, self.page_table)
+        self.idx = torch.full((2, layers, S, w.Hkv, w.kmax), -1, dtype=torch.int32, device=dev)
+        self.cnt = torch.zeros((2, layers, S, w.Hkv), dtype=torch.int32, device=dev)
+        self.o_sel = torch.empty((layers, *w.q1.shape), dtype=torch.bfloat16, device=dev)
+        self.o_sp = torch.empty((layers, *w.q1.shape), dtype=torch.bfloat16, device=dev)
+        self.ws_sel = dsa.Workspace(dsa.select_workspace_size(self.dims), dev)
+        self.ws_sp = dsa.Workspace(dsa.sparse_workspace_size(self.dims), dev)
+        self.host_o = torch.empty((T, *w.q1.shape), dtype=torch.bfloat16).pin_memory()
+        self.host_idx = torch.empty((w.S, w.Hkv, w.kmax), dtype=torch.int32).pin_memory()
+
+    # one call each -------------------------------------------------------------
+    def select(self, l, buf, stream):
+        self.dsa.dsa_select(self.q[l, 0], self.k[l], self.v[l], self.n_ctx, self.w.P, self.topk,
+                            self.idx[buf, l], self.o_sel[l], stream, dims=self.dims,
+                            cnt_out=self.cnt[buf, l], workspace=self.ws_sel)
+
+    def sparse(self, l, t, buf, stream):
+        self.dsa.dsa_sparse_attn(self.q[l, t], self.k[l], self.v[l], self.idx[buf, l],
+                                 self.bk[l, t], self.bv[l, t], self.o_sp[l], stream,
+                                 dims=self.dims, n_ctx=self.n_ctx, idx_cnt=self.cnt[buf, l],
+                                 workspace=self.ws_sp)
+
+    # the block step: select(next) on the side stream || sparse(current) on main
+    def block_step(self, cur, e2e=False):
+        nxt = 1 - cur
+        self.side.wait_stream(self.main)
+        with torch.cuda.stream(self.side):
+            for l in range(self.L):
+                if e2e:
+                    self.q[l, 0].copy_(self.host_q[0], non_blocking=True)
+                self.select(l, nxt, self.side)
+                if e2e:
+                    self.host_o[0].copy_(self.o_sel[l], non_blocking=True)
+                    self.host_idx.copy_(self.idx[nxt, l], non_blocking=True)
+        for t in range(1, self.w.T):
+            for l in range(self.L):
+                if e2e:
+                    self.q[l, t].copy_(self.host_q[t], non_blocking=True)
+                    self.bk[l, t].copy_(self.host_bk[t], non_blocking=True)
+                    self.bv[l, t].copy_(self.host_bv[t], non_blocking=True)
+                self.sparse(l, t, cur, self.main)
+                if e2e:
+                    self.host_o[t].copy_(self.o_sp[l], non_blocking=True)
+        self.main.wait_stream(self.side)
+
+    def h2d_d2h_bytes(self):
+        w, L = self.w, self.L
+        q = self.host_q[0].numel() * 2
+        blk = self.host_bk[0].numel() * 2
+        h2d = L * (q + (w.T - 1) * (q + 2 * blk))
+        d2h = L * (q + self.host_idx.numel() * 4 + (w.T - 1) * q)
+        return h2d, d2h
+
+    def capture(self, e2e=False):
+        graphs = []
+        for cur in (0, 1):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.main, capture_error_mode="relaxed"):
+                self.block_step(cur, e2e)
+            graphs.append(g)
+        return graphs
+
+    def capture_sparse_only(self):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.main, capture_error_mode="relaxed"):
+            for t in range(1, self.w.T):
+                for l in range(self.L):
+                    self.sparse(l, t, 0, self.main)
+        return g
+
+
+def timed(fn, reps, stream):
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(reps):
+        fn(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / reps  # ms
+
+
+def run_ours(args, world, rank, local):
+    from block_sparse_attention_27_b200 import build as build_mod
+    from block_sparse_attention_27_b200 import dsa
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the CUDA library has no CPU path)")
+    build_mod.build()
+    dsa.load()
+    torch.cuda.set_device(local)
+    main_stream = torch.cuda.Stream()   # graphs cannot be captured on the legacy stream
+    with torch.cuda.stream(main_stream):
+        _run_ours(args, world, rank, local, dsa)
+
+
+def _run_ours(args, world, rank, local, dsa):
+    w = W.make(args.workload, 0)
+    b = Bench(w, args.layers, dsa)
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+    T, L = w.T, args.layers
+    step_bytes = L * (select_bytes(w) + (T - 1) * sparse_bytes(w))
+    launches_per_step = L * (dsa.kernels_per_call(0) + (T - 1) * dsa.kernels_per_call(1))
+
+    # initial selection (block 0's indices), eager warm-up of every kernel
+    for l in range(L):
+        b.select(l, 0, b.main)
+    b.sparse(0, 1, 0, b.main)
+    torch.cuda.synchronize()
+
+    graphs = b.capture()
+    for i in range(args.warmup):
+        graphs[i % 2].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = timed(lambda i: graphs[(args.warmup + i) % 2].replay(), args.steps, b.main)
+    barrier(world)
+    ms = max_over_ranks(ms, world)
+    status_sel, status_sp = b.ws_sel.status(), b.ws_sp.status()
+    if status_sel != dsa.DSA_OK or status_sp != dsa.DSA_OK:
+        raise SystemExit(f"device status: select {status_sel}, sparse {status_sp}")
+
+    # phase timings (reported beside the headline): selection alone, sparse alone
+    reps = 3
+    sel_ms = timed(lambda i: [b.select(l, 0, b.main) for l in range(L)], reps, b.main) / L
+    g_sp = b.capture_sparse_only()
+    g_sp.replay()
+    sp_us = 1e3 * timed(lambda i: g_sp.replay(), reps, b.main) / ((T - 1) * L)
+    del g_sp
+
+    # e2e: the same step with host<->device copies of every call's inputs/outputs
+    e2e_graphs = b.capture(e2e=True)
+    for i in range(2):
+        e2e_graphs[i % 2].replay()
+    e2e_ms = max_over_ranks(timed(lambda i: e2e_graphs[i % 2].replay(), args.steps, b.main), world)
+    del e2e_graphs
+    h2d, d2h = b.h2d_d2h_bytes()
+
+    if rank != 0:
+        return
+    sel_b, sp_b = select_bytes(w), sparse_bytes(w)
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    sel_gbs = sel_b / (sel_ms * 1e-3) / 1e9
+    sp_gbs = sp_b / (sp_us * 1e-6) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT.get(args.workload, args.workload),
+                   "step": f"one denoising block over {L} independent layer copies: selection "
+                           f"of the next block ({L} x dsa_select, second stream) overlapped with "
+                           f"{T - 1} x {L} dsa_sparse_attn of the current block",
+                   "layers_rotated": L,
+                   "l2": f"inputs larger than L2: {L} distinct K/V caches, queries and outputs "
+                         f"({step_bytes / 1e9:.1f} GB of algorithmic traffic per step)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "sparse_step_us": round(sp_us, 3),
+        "sparse_step_gbs": round(sp_gbs, 1),
+        "select_pass_ms": round(sel_ms, 4),
+        "select_pass_gbs": round(sel_gbs, 1),
+        "roofline": {"bound": "hbm", "kernel": "selection pass (dsa_select)",
+                     "achieved": round(sel_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(sel_gbs / hbm_peak, 4),
+                     "traffic": recorded_traffic("select", args.workload),
+                     "algorithmic_bytes_per_launch": sel_b, "peak_kind": peak_kind},
+        "roofline_sparse": {"bound": "hbm", "kernel": "sparse step (dsa_sparse_attn)",
+                            "achieved": round(sp_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                            "frac": round(sp_gbs / hbm_peak, 4),
+                            "traffic": recorded_traffic("sparse", args.workload),
+                            "algorithmic_bytes_per_launch": sp_b, "peak_kind": peak_kind},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "clocks": clk.summary(),
+        "tensor_tflops_select": round(select_flops(w) / (sel_ms * 1e-3) / 1e12, 1),
+        "tensor_peak_tflops": tc_peak,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line, ensure_ascii=False), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="128k", choices=list(WORKLOAD_TEXT))
+    ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        # the oracle needs no GPU and no process group: rank 0 runs, the others exit
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
+                      int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

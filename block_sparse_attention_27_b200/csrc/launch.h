@@ -1,0 +1,71 @@
+// launch.h -- internal interface between the C-ABI host code (api.cu) and the
+// kernel files.  Not installed; the public interface is include/dsa.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dsa {
+
+// Shape of one call, resolved on the host.
+struct Shape {
+  int S, B, Hq, Hkv, G, BG, d, P, max_pages, kmax;
+  long long n_phys;
+  const int32_t *page_table;  // may be null (identity)
+  float sl2;                  // log2(e) / sqrt(d)
+};
+
+// Kernel launches issued by one dsa_select / dsa_sparse_attn call.
+constexpr int kSelectLaunches = 3;
+constexpr int kSparseLaunches = 2;
+
+// ---- selection pass ----
+struct SelectPlan {
+  int rowtiles;         // ceil(BG / 128)
+  int splits;           // key splits per (seq, KV head, row tile)
+  int tiles_per_split;  // 64-token tiles per split
+  int max_tiles;        // ceil(max_pages * P / 64)
+  size_t off_part_o, off_part_ml, off_pagepart, off_mtile, off_scores, total;
+};
+
+struct SelectArgs {
+  const __nv_bfloat16 *q, *k, *v;
+  const int32_t *n_ctx, *topk;
+  int32_t *idx_out, *cnt_out;
+  __nv_bfloat16 *o_out;
+  float *part_o;    // [S, Hkv, rowtiles*splits... ] see select.cu
+  float *part_ml;
+  float *pagepart;  // [S, Hkv, max_pages, BG]
+  float *mtile;     // [S, Hkv, max_tiles, BG]
+  float *scores;    // [S, Hkv, max_pages]
+  uint32_t *status;
+};
+
+SelectPlan plan_select(const Shape &sh, int num_sms);
+cudaError_t launch_select(const Shape &sh, const SelectPlan &plan, const SelectArgs &a,
+                          cudaStream_t stream);
+
+// ---- sparse pass ----
+struct SparsePlan {
+  int rowtiles;
+  int sel_tiles;  // ceil(kmax * P / 64): 64-key tiles over the selected pages
+  int blk_tiles;  // ceil(B / 64): tiles over the block's own tokens
+  int ntiles;     // sel_tiles + blk_tiles
+  size_t off_part_o, off_part_ml, total;
+};
+
+struct SparseArgs {
+  const __nv_bfloat16 *q, *k, *v, *blk_k, *blk_v;
+  const int32_t *idx, *idx_cnt, *n_ctx;
+  __nv_bfloat16 *o_out;
+  float *part_o;   // [S, Hkv, ntiles, BG, d]
+  float *part_ml;  // [S, Hkv, ntiles, BG, 2]
+  uint32_t *status;
+};
+
+SparsePlan plan_sparse(const Shape &sh, int num_sms);
+cudaError_t launch_sparse(const Shape &sh, const SparsePlan &plan, const SparseArgs &a,
+                          cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,159 @@
+/*
+ * dsa.h -- C ABI of libdsa: shared-index top-k sparse KV attention for
+ * block-diffusion LLMs on NVIDIA B200 (sm_100a).
+ *
+ * The method ("MAGE: All-[MASK] Block Already Knows Where to Look in Block
+ * Diffusion LLM"): all B query tokens of a denoising block share ONE set of KV
+ * pages per KV head (Problem section).  Step 1 of the block runs one exact
+ * attention pass over the whole prefix and keeps the top-k pages (Approach:
+ * selection), every later denoising step attends only to those pages plus the
+ * block's own tokens, reusing the step-1 indices (Approach: reuse).  Selection is
+ * meant to run on a second CUDA stream (Approach: "async CUDA stream").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Element types: q/k/v/blk_k/blk_v/o are bf16 (2-byte IEEE bfloat16); index
+ *  arrays are int32.  Every pointer passed here is a DEVICE pointer unless the
+ *  argument says "host".  The caller owns all memory; the library allocates
+ *  nothing and keeps no state except a per-device cache of the SM count.
+ *
+ *  Layouts (row-major, innermost last):
+ *    q_blk        [S, B, Hq, d]          queries of the block (post-RoPE)
+ *    k_cache      [n_phys, Hkv, page, d] paged key cache
+ *    v_cache      [n_phys, Hkv, page, d] paged value cache
+ *    page_table   [S, max_pages]         logical page -> physical page (int32);
+ *                                        NULL = identity, physical = s*max_pages + lp
+ *    n_ctx        [S]                    prefix length of each sequence (tokens)
+ *    topk         [S]                    page budget of each sequence in TOKENS,
+ *                                        a multiple of `page`
+ *    idx          [S, Hkv, kmax]         selected LOGICAL pages, ascending, -1 padded
+ *    idx_cnt      [S, Hkv]               number of valid entries of each idx row
+ *    blk_k, blk_v [S, B, Hkv, d]         the block's own keys / values
+ *    o_out        [S, B, Hq, d]          attention output (bf16)
+ *  Query head j uses KV head j / (Hq/Hkv) (contiguous GQA groups).  The softmax
+ *  scale is 1/sqrt(d).  A prefix token t of sequence s lives in logical page
+ *  t / page, slot t % page; tokens t >= n_ctx[s] of the last page are ignored.
+ *
+ *  Alignment: q_blk, k_cache, v_cache, blk_k, blk_v and o_out must be 16-byte
+ *  aligned.  Supported shapes: d in {64, 128}; page in {16, 32, 64};
+ *  Hq % Hkv == 0; B * Hq/Hkv <= 256; kmax >= 1 (it may exceed the pages of a
+ *  prefix: the extra entries are -1).
+ *
+ *  Return values: 0 on success, or a negative DSA_ERR_* code.  Argument errors
+ *  are detected on the host before anything is launched.  All work is queued
+ *  asynchronously on `stream`; no call synchronises except dsa_get_status().
+ *  Errors found by the kernels (a bad page index, a page-table entry outside the
+ *  cache, non-finite scores, a device wait that gave up) never fault: the kernel
+ *  skips the offending access, finishes, and sets a bit in the status word at
+ *  the start of the workspace, which dsa_get_status() reads.
+ *
+ *  Workspace: each call takes a caller-owned device workspace of at least
+ *  dsa_*_workspace_size() bytes.  Zero it once with dsa_workspace_init() after
+ *  allocation.  Calls that may run concurrently (the selection pass on one stream
+ *  and sparse steps on another) need separate workspaces.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes (negative).  The first four are returned synchronously; the last
+ * three are reported through the workspace status word. */
+#define DSA_OK 0
+#define DSA_ERR_INVALID_ARG (-1)        /* null/misaligned pointer, bad shape or value */
+#define DSA_ERR_UNSUPPORTED (-2)        /* valid but outside the supported shapes */
+#define DSA_ERR_WORKSPACE_TOO_SMALL (-3)
+#define DSA_ERR_CUDA (-4)               /* a CUDA launch or runtime call failed */
+#define DSA_ERR_DEVICE_TIMEOUT (-5)     /* a bounded device wait gave up */
+#define DSA_ERR_BAD_INDEX (-6)          /* idx entry >= number of pages, or page-table entry outside the cache */
+#define DSA_ERR_NONFINITE (-7)          /* a page score was NaN or Inf (non-finite inputs) */
+
+typedef struct dsa_dims {
+  int32_t S;          /* sequences in the batch */
+  int32_t B;          /* query tokens per block */
+  int32_t Hq;         /* query heads */
+  int32_t Hkv;        /* KV heads; Hq % Hkv == 0 */
+  int32_t d;          /* head dimension (64 or 128) */
+  int32_t page;       /* tokens per KV page (16, 32 or 64) */
+  int32_t max_pages;  /* length of a page-table row: logical pages per sequence, upper bound */
+  int32_t kmax;       /* length of an idx row: selected pages per (sequence, KV head), upper bound */
+  int64_t n_phys;     /* physical pages held by k_cache / v_cache */
+  const int32_t *page_table; /* device [S, max_pages] or NULL (identity) */
+} dsa_dims;
+
+/* cudaStream_t without including the CUDA headers. */
+typedef struct CUstream_st *dsa_stream_t;
+
+/*
+ * Selection pass (MAGE page, Approach): exact attention of the block's step-1
+ * queries over the whole prefix of every sequence.
+ *   - o_out receives, for each query row, softmax(q K^T / sqrt(d)) V over the
+ *     prefix tokens only (the block's own tokens are not part of this pass).
+ *   - For each (sequence, KV head) the attention probabilities are averaged over
+ *     the B queries and the G = Hq/Hkv query heads of the group, summed inside
+ *     each page, and the kp = topk[s]/page pages with the largest sums are kept;
+ *     on equal sums the lower page index wins.  idx_out receives them in
+ *     ascending order, padded with -1; cnt_out receives min(kp, pages of the
+ *     prefix).  Requires topk[s]/page <= kmax.
+ * Arguments: q_blk, k_cache, v_cache (bf16, layouts above); n_ctx (device int32
+ * [S]); page (must equal dims->page); topk (DEVICE int32 [S], tokens); idx_out
+ * (device int32 [S,Hkv,kmax]); o_out (device bf16 [S,B,Hq,d]); stream; dims;
+ * cnt_out (device int32 [S,Hkv]); workspace/ws_bytes (device, see above).
+ */
+int dsa_select(const void *q_blk, const void *k_cache, const void *v_cache,
+               const int32_t *n_ctx, int32_t page, const int32_t *topk,
+               int32_t *idx_out, void *o_out, dsa_stream_t stream,
+               const dsa_dims *dims, int32_t *cnt_out,
+               void *workspace, size_t ws_bytes);
+
+/*
+ * Sparse pass, denoising steps 2..T (MAGE page, Approach: the step-1 indices are
+ * reused for every later step).  For each query row (b, j) of sequence s:
+ * softmax attention, scale 1/sqrt(d), over the key set
+ *   { prefix tokens t < n_ctx[s] of the pages idx[s, j/G, 0 .. idx_cnt-1] }
+ *   U { the block's own tokens u = 0..B-1 with keys blk_k[s,u,j/G], values blk_v[s,u,j/G] }
+ * with no mask inside the block (bidirectional, self included).  idx entries
+ * must be distinct logical pages below ceil(n_ctx[s]/page); an entry outside
+ * that range is skipped and reported as DSA_ERR_BAD_INDEX through the status word.
+ */
+int dsa_sparse_attn(const void *q_blk, const void *k_cache, const void *v_cache,
+                    const int32_t *idx, const void *blk_k, const void *blk_v,
+                    void *o_out, dsa_stream_t stream,
+                    const dsa_dims *dims, const int32_t *n_ctx, const int32_t *idx_cnt,
+                    void *workspace, size_t ws_bytes);
+
+/* Workspace bytes each pass needs for `dims` on the current CUDA device
+ * (0 if dims is invalid). */
+size_t dsa_select_workspace_size(const dsa_dims *dims);
+size_t dsa_sparse_workspace_size(const dsa_dims *dims);
+
+/* Zeroes the status word and counters of a freshly allocated workspace
+ * (asynchronous on `stream`). */
+int dsa_workspace_init(void *workspace, size_t ws_bytes, dsa_stream_t stream);
+
+/* Synchronises `stream`, reads the workspace status word and returns DSA_OK or
+ * the most severe device-side code recorded since dsa_workspace_init(); the word
+ * is left as it is (sticky).  Returns DSA_ERR_CUDA if the read fails. */
+int dsa_get_status(const void *workspace, dsa_stream_t stream);
+
+/* Static description of a status code. */
+const char *dsa_strerror(int code);
+
+/* Number of kernel launches one call issues on its stream: pass 0 = dsa_select,
+ * pass 1 = dsa_sparse_attn (DSA_ERR_INVALID_ARG otherwise).  Useful when
+ * capturing calls into a CUDA graph or counting launches. */
+int dsa_kernels_per_call(int pass);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

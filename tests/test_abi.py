@@ -1,0 +1,103 @@
+"""The C-ABI library loads, exports every symbol include/dsa.h declares, and rejects
+bad arguments on the host before touching a GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_27_b200 import build as B
+from block_sparse_attention_27_b200 import dsa
+
+HEADER = os.path.join(B.ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return dsa.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(dsa.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_strerror_and_version(lib):
+    assert lib.dsa_version() >= 100
+    assert dsa.kernels_per_call(0) >= 1 and dsa.kernels_per_call(1) >= 1
+    assert lib.dsa_kernels_per_call(7) == dsa.DSA_ERR_INVALID_ARG
+    for code in range(0, -8, -1):
+        assert dsa.strerror(code) and "unknown" not in dsa.strerror(code)
+    assert "unknown" in dsa.strerror(-99)
+
+
+def good_dims(**kw):
+    base = dict(S=1, B=32, Hq=32, Hkv=8, d=128, page=16, max_pages=512, kmax=32, n_phys=512)
+    base.update(kw)
+    return dsa.make_dims(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=30), dsa.DSA_ERR_INVALID_ARG),      # Hq % Hkv != 0
+    (dict(d=96), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(page=8), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(B=65, Hq=32, Hkv=8), dsa.DSA_ERR_UNSUPPORTED),  # B*G = 260 > 256
+    (dict(kmax=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(S=0), dsa.DSA_ERR_INVALID_ARG),
+])
+def test_bad_dims_rejected_on_host(lib, kw, code):
+    dims = good_dims(**kw)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    rc = lib.dsa_select(fake, fake, fake, fake, dims.page, fake, fake, fake, None,
+                        ctypes.byref(dims), fake, fake, 1 << 30)
+    assert rc == code
+    assert lib.dsa_select_workspace_size(ctypes.byref(dims)) == 0
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    dims = good_dims()
+    ok = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    rc = lib.dsa_select(None, ok, ok, ok, 16, ok, ok, ok, None, ctypes.byref(dims), ok, ok, 1 << 30)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+    rc = lib.dsa_select(bad, ok, ok, ok, 16, ok, ok, ok, None, ctypes.byref(dims), ok, ok, 1 << 30)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+    rc = lib.dsa_select(ok, ok, ok, ok, 32, ok, ok, ok, None, ctypes.byref(dims), ok, ok, 1 << 30)
+    assert rc == dsa.DSA_ERR_INVALID_ARG  # page argument disagrees with dims
+    rc = lib.dsa_sparse_attn(ok, ok, ok, ok, ok, bad, ok, None, ctypes.byref(dims), ok, ok, ok,
+                             1 << 30)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_workspace_too_small_rejected(lib):
+    dims = good_dims()
+    ok = ctypes.c_void_p(1 << 20)
+    need = lib.dsa_sparse_workspace_size(ctypes.byref(dims))
+    assert need > 4096
+    rc = lib.dsa_sparse_attn(ok, ok, ok, ok, ok, ok, ok, None, ctypes.byref(dims), ok, ok, ok,
+                             need - 1)
+    assert rc == dsa.DSA_ERR_WORKSPACE_TOO_SMALL
+    need = lib.dsa_select_workspace_size(ctypes.byref(dims))
+    rc = lib.dsa_select(ok, ok, ok, ok, 16, ok, ok, ok, None, ctypes.byref(dims), ok, ok, need - 1)
+    assert rc == dsa.DSA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_library_has_no_oracle_dependency():
+    """The product library is built from csrc/ only and never references the oracle."""
+    for src in os.listdir(os.path.join(B.PKG, "csrc")):
+        text = open(os.path.join(B.PKG, "csrc", src)).read()
+        assert "oracle" not in text.lower(), src
+    for py in ("dsa.py", "build.py", "__init__.py"):
+        text = open(os.path.join(B.PKG, py)).read()
+        assert "import oracle" not in text and "from oracle" not in text

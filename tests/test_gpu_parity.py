@@ -1,0 +1,159 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from block_sparse_attention_27_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa_mod():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for -m gpu tests")
+    from block_sparse_attention_27_b200 import build, dsa
+    build.build()
+    dsa.load()
+    return dsa
+
+
+# name -> (workload, overrides); sizes span several tiles and ragged tails
+CASES = {
+    "tiny": ("tiny", {}),
+    "tiny_tail_d64": ("tiny", dict(n=1000, topk=96)),
+    "8k": ("8k", {}),
+    "32k_g7_p64": ("32k", {}),
+    "small_g7_p64_tail": ("32k", dict(n=5000, topk=512)),
+    "ragged_paged": ("batched", dict(S=3, n_lo=100, n_hi=3000, B=8, Hq=8, Hkv=2,
+                                     topk_choices=(64, 128, 4096))),
+    "b1": ("8k", dict(n=3000, B=1, topk=256)),
+    "kp1": ("8k", dict(n=2000, topk=16)),
+    "budget_covers_prefix": ("8k", dict(n=1500, topk=2048)),
+    "p32": ("8k", dict(n=4000, P=32, topk=512)),
+    "p64_d64": ("tiny", dict(n=3000, P=64, topk=256, B=8, Hq=8, Hkv=2)),
+}
+
+
+def kp_list(w):
+    return [int(w.topk[s]) // w.P for s in range(w.S)]
+
+
+def run_case(dsa_mod, w, steps=(2,)):
+    dw = dsa_mod.DeviceWorkload(w)
+    dw.select()
+    torch.cuda.synchronize()
+    assert dw.ws_sel.status() == dsa_mod.DSA_OK
+    pt = None if w.page_table is None else w.page_table.numpy()
+    ref = oracle.select(W.bits(w.q1), W.bits(w.k_cache), W.bits(w.v_cache), w.n_ctx.numpy(),
+                        w.topk.numpy(), page_table=pt, max_pages=w.max_pages)
+    gidx, gcnt = dw.idx.cpu().numpy(), dw.cnt.cpu().numpy()
+    parity.check_selection(gidx, gcnt, ref, [w.n_pages(s) for s in range(w.S)], kp_list(w))
+    parity.check_output(dw.o_sel, ref.o, f"{w.name} selection o_out")
+    for t in steps:
+        q, bk, bv = w.step_inputs(t)
+        o = dw.sparse(q.cuda(), bk.cuda(), bv.cuda())
+        torch.cuda.synchronize()
+        assert dw.ws_sp.status() == dsa_mod.DSA_OK
+        ref_o, _ = oracle.sparse(W.bits(q), W.bits(w.k_cache), W.bits(w.v_cache), w.n_ctx.numpy(),
+                                 gidx, gcnt, W.bits(bk), W.bits(bv), page_table=pt,
+                                 max_pages=w.max_pages)
+        parity.check_output(o, ref_o, f"{w.name} sparse step {t}")
+    return dw, ref
+
+
+@pytest.mark.parametrize("case", list(CASES), ids=list(CASES))
+def test_parity(dsa_mod, case):
+    name, kw = CASES[case]
+    run_case(dsa_mod, W.make(name, 0, **kw), steps=(2, 3))
+
+
+@pytest.mark.parametrize("name", ["128k", "batched"])
+def test_parity_full_size(dsa_mod, name):
+    """Full-size workloads in the launch configuration the bench times."""
+    run_case(dsa_mod, W.make(name, 0), steps=(2,))
+
+
+def test_planted_needles_selected(dsa_mod):
+    w = W.make("tiny", 0)
+    dw = dsa_mod.DeviceWorkload(w)
+    dw.select()
+    assert dw.idx[0, 0].cpu().tolist() == w.planted[(0, 0)]
+
+
+def test_exact_ties_resolved_within_window(dsa_mod):
+    w = W.make("8k", 1, n=2048, topk=256)
+    for b, a in ((40, 3), (77, 10), (100, 64)):      # bit-identical page copies
+        w.k_cache[b] = w.k_cache[a]
+        w.v_cache[b] = w.v_cache[a]
+    run_case(dsa_mod, w)
+
+
+def test_dense_when_budget_covers_prefix(dsa_mod):
+    """kp >= pages: the sparse pass is dense attention over prefix + block."""
+    w = W.make("8k", 2, n=1200, topk=2048)
+    dw, _ = run_case(dsa_mod, w)
+    idx, cnt = oracle.all_pages(w.n_ctx.numpy(), w.P, w.Hkv, kmax=w.kmax)
+    assert np.array_equal(dw.idx.cpu().numpy(), idx)
+
+
+def test_bad_index_reported_not_faulting(dsa_mod):
+    w = W.make("8k", 3, n=1000, topk=128)
+    dw = dsa_mod.DeviceWorkload(w)
+    dw.select()
+    idx = dw.idx.clone()
+    idx[0, 0, 0] = w.n_pages(0) + 5      # past the prefix
+    idx[0, 1, 1] = -7
+    q, bk, bv = w.step_inputs(2)
+    dw.sparse(q.cuda(), bk.cuda(), bv.cuda(), idx=idx)
+    torch.cuda.synchronize()
+    assert dw.ws_sp.status() == dsa_mod.DSA_ERR_BAD_INDEX
+    assert torch.isfinite(dw.o_sp.float()).all()
+
+
+def test_nonfinite_input_reported(dsa_mod):
+    w = W.make("8k", 4, n=1000, topk=128)
+    w.q1[0, 0, 0, 0] = float("nan")
+    dw = dsa_mod.DeviceWorkload(w)
+    dw.select()
+    torch.cuda.synchronize()
+    assert dw.ws_sel.status() == dsa_mod.DSA_ERR_NONFINITE
+
+
+def test_selection_on_second_stream(dsa_mod):
+    """Selection on a side stream, gated to the sparse stream by an event, gives the
+    same indices and outputs as running everything on one stream."""
+    w = W.make("8k", 5, n=6000)
+    dw = dsa_mod.DeviceWorkload(w)
+    q, bk, bv = (x.cuda() for x in w.step_inputs(2))
+    dw.select()
+    o_ref = dw.sparse(q, bk, bv).clone()
+    idx_ref = dw.idx.clone()
+    dw.idx.fill_(-1)
+    side = torch.cuda.Stream()
+    ev = torch.cuda.Event()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        dw.select(stream=side)
+        ev.record(side)
+    torch.cuda.current_stream().wait_event(ev)
+    o = dw.sparse(q, bk, bv)
+    torch.cuda.synchronize()
+    assert torch.equal(dw.idx, idx_ref)
+    assert torch.equal(o, o_ref)
+
+
+def test_deterministic(dsa_mod):
+    w = W.make("8k", 6, n=5000)
+    dw = dsa_mod.DeviceWorkload(w)
+    q, bk, bv = (x.cuda() for x in w.step_inputs(2))
+    dw.select()
+    a = (dw.idx.clone(), dw.o_sel.clone(), dw.sparse(q, bk, bv).clone())
+    dw.select()
+    b = (dw.idx.clone(), dw.o_sel.clone(), dw.sparse(q, bk, bv).clone())
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
