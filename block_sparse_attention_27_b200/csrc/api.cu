@@ -185,8 +185,6 @@ int dsa_sparse_attn(const void *q_blk, const void *k_cache, const void *v_cache,
   a.idx_cnt = idx_cnt;
   a.n_ctx = n_ctx;
   a.o_out = static_cast<__nv_bfloat16 *>(o_out);
-  a.part_o = at<float>(workspace, plan.off_part_o);
-  a.part_ml = at<float>(workspace, plan.off_part_ml);
   a.status = at<uint32_t>(workspace, 0);
   if (dsa::launch_sparse(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DSA_ERR_CUDA;

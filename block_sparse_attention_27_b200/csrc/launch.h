@@ -2,6 +2,7 @@
 // kernel files.  Not installed; the public interface is include/dsa.h.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -16,9 +17,19 @@ struct Shape {
   float sl2;                  // log2(e) / sqrt(d)
 };
 
+// TMA map of a paged cache [n_phys, Hkv, P, D] viewed as rows of D bf16; boxes of
+// box_rows rows x 64 elements with the 128-byte swizzle (tmap.cu).
+cudaError_t make_kv_tensor_map(CUtensorMap *out, const void *base, long long rows, int D,
+                               int box_rows);
+
+// The block's own keys/values [S*B, Hkv, D] bf16; boxes of 64 elements x 1 head x
+// 64 tokens with the 128-byte swizzle (tmap.cu).
+cudaError_t make_blk_tensor_map(CUtensorMap *out, const void *base, long long tokens, int Hkv,
+                                int D);
+
 // Kernel launches issued by one dsa_select / dsa_sparse_attn call.
 constexpr int kSelectLaunches = 3;
-constexpr int kSparseLaunches = 2;
+constexpr int kSparseLaunches = 1;
 
 // ---- selection pass ----
 struct SelectPlan {
@@ -48,19 +59,17 @@ cudaError_t launch_select(const Shape &sh, const SelectPlan &plan, const SelectA
 
 // ---- sparse pass ----
 struct SparsePlan {
-  int rowtiles;
-  int sel_tiles;  // ceil(kmax * P / 64): 64-key tiles over the selected pages
-  int blk_tiles;  // ceil(B / 64): tiles over the block's own tokens
-  int ntiles;     // sel_tiles + blk_tiles
-  size_t off_part_o, off_part_ml, total;
+  int rowtiles;   // ceil(BG / 128)
+  int cluster;    // CTAs per (seq, KV head, row tile): one thread-block cluster
+  int ppc;        // selected pages per CTA of the cluster
+  int blk_tiles;  // ceil(B / 64): tiles over the block's own tokens (last CTA)
+  size_t total;   // workspace bytes (status word)
 };
 
 struct SparseArgs {
   const __nv_bfloat16 *q, *k, *v, *blk_k, *blk_v;
   const int32_t *idx, *idx_cnt, *n_ctx;
   __nv_bfloat16 *o_out;
-  float *part_o;   // [S, Hkv, ntiles, BG, d]
-  float *part_ml;  // [S, Hkv, ntiles, BG, 2]
   uint32_t *status;
 };
 

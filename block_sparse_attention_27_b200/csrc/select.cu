@@ -16,14 +16,14 @@
 //      ties broken towards the lower page index, emitted in ascending order.
 #include <algorithm>
 
-#include "attn_core.cuh"
 #include "launch.h"
+#include "sm100.cuh"
+#include "tc_attn.cuh"
 
 namespace dsa {
 namespace {
 
-constexpr int kSelThreads = 256;  // 8 warps
-constexpr int kRowsPerCta = 128;
+constexpr int kRowsPerCta = 128;  // query rows per CTA (one M=128 MMA tile)
 
 struct PartialParams {
   Shape sh;
@@ -31,131 +31,136 @@ struct PartialParams {
   SelectArgs a;
 };
 
+// ---------------------------------------------------------------------------
+// select_partial: tcgen05 split-KV attention (tc_attn.cuh engine) over the
+// split's contiguous 64-token tiles of the prefix, loaded page by page through
+// the page table.  After each tile the softmax threads record, per (page, row),
+// the tile's probability mass relative to the row's reference max (pagepart)
+// and that max (mtile); the split's unnormalised O row, m and l go to part_o /
+// part_ml.
+// ---------------------------------------------------------------------------
+constexpr int kSelStages = 4;
+
 template <int D, int PAGE>
-__global__ void __launch_bounds__(kSelThreads, 2) select_partial(const PartialParams pp) {
-  extern __shared__ __align__(128) unsigned char smem[];
+struct SelectPolicy {
+  const Shape *sh;
+  const SelectPlan *plan;
+  const SelectArgs *a;
+  const CUtensorMap *kmap, *vmap;
+  int s, h, n, np, t_begin, row_base;
+  size_t sh_idx;
+  float sl2;
+
+  __device__ __forceinline__ long long phys_of(int lp) const {
+    if (lp >= np) return -1;
+    const long long p = sh->page_table ? (long long)sh->page_table[(size_t)s * sh->max_pages + lp]
+                                       : (long long)s * sh->max_pages + lp;
+    return (p >= 0 && p < sh->n_phys) ? p : -1;
+  }
+  __device__ __forceinline__ void prefetch() const {
+    sm100::tma_prefetch_map(kmap);
+    sm100::tma_prefetch_map(vmap);
+  }
+  __device__ __forceinline__ void load_tile(int k, uint32_t sk, uint32_t sv, uint32_t half_bytes,
+                                            uint32_t bar) const {
+    constexpr int kPages = tc::kBN / PAGE;
+    const int lp0 = (t_begin + k) * tc::kBN / PAGE;
+    long long phys[kPages];
+    uint32_t nvalid = 0;
+#pragma unroll
+    for (int pi = 0; pi < kPages; ++pi) {
+      phys[pi] = phys_of(lp0 + pi);
+      if (phys[pi] >= 0) ++nvalid;
+      else if (lp0 + pi < np && blockIdx.x == 0) raise_status(a->status, kStatusBadIndex);
+    }
+    sm100::mbar_arrive_expect_tx(bar, nvalid * PAGE * 128u * (D / 64) * 2u);
+#pragma unroll
+    for (int pi = 0; pi < kPages; ++pi) {
+      if (phys[pi] < 0) continue;
+      const int y = (int)((phys[pi] * sh->Hkv + h) * PAGE);
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        sm100::tma_load_2d(sk + hf * half_bytes + pi * PAGE * 128, kmap, bar, hf * 64, y);
+        sm100::tma_load_2d(sv + hf * half_bytes + pi * PAGE * 128, vmap, bar, hf * 64, y);
+      }
+    }
+  }
+  __device__ __forceinline__ const __nv_bfloat16 *q_row(int r) const {
+    const int row = row_base + r;
+    if (row >= sh->BG) return nullptr;
+    const int b = row / sh->G, g = row % sh->G;
+    return a->q + (((size_t)s * sh->B + b) * sh->Hq + (size_t)h * sh->G + g) * D;
+  }
+  __device__ __forceinline__ uint64_t key_mask(int k) const {
+    const int t0 = (t_begin + k) * tc::kBN;
+    uint64_t m = 0;
+#pragma unroll
+    for (int pi = 0; pi < tc::kBN / PAGE; ++pi) {
+      if (phys_of(t0 / PAGE + pi) < 0) continue;
+      const int lo = t0 + pi * PAGE;
+      const int cnt = min(PAGE, n - lo);
+      if (cnt > 0) m |= ((cnt >= 64) ? ~0ull : ((1ull << cnt) - 1ull)) << (pi * PAGE);
+    }
+    return m;
+  }
+  __device__ __forceinline__ void after_tile(int k, int r, float m_used, const float *psum) const {
+    const int row = row_base + r;
+    if (row >= sh->BG) return;
+    const int tile = t_begin + k;
+    a->mtile[(sh_idx * plan->max_tiles + tile) * sh->BG + row] = m_used;
+#pragma unroll
+    for (int pi = 0; pi < tc::kBN / PAGE; ++pi) {
+      const int lp = tile * tc::kBN / PAGE + pi;
+      if (lp < np) a->pagepart[(sh_idx * sh->max_pages + lp) * sh->BG + row] = psum[pi];
+    }
+  }
+};
+
+template <int D, int PAGE>
+__global__ void __launch_bounds__(tc::kThreads, 1)
+    select_partial(const PartialParams pp, const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap) {
+  extern __shared__ unsigned char smem_raw[];
   const Shape &sh = pp.sh;
   const SelectPlan &plan = pp.plan;
   const SelectArgs &a = pp.a;
-  constexpr int kTileBytes = kKeyTile * D * 2;
-  unsigned char *sQ = smem;
-  unsigned char *sKV = smem + kRowsPerCta * D * 2;  // [stage][K|V] tiles
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int s = blockIdx.z, h = blockIdx.y;
   const int split = blockIdx.x / plan.rowtiles, rt = blockIdx.x % plan.rowtiles;
   const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status,
-                             tid == 0 && blockIdx.x == 0);
-  const int np = (n + PAGE - 1) / PAGE;
-  const int ntiles = (n + kKeyTile - 1) / kKeyTile;
+                             threadIdx.x == 0 && blockIdx.x == 0);
+  const int ntiles = (n + tc::kBN - 1) / tc::kBN;
   const int t_begin = split * plan.tiles_per_split;
-  const int t_end = min(ntiles, t_begin + plan.tiles_per_split);
-  const int row_base = rt * kRowsPerCta;
-  const int warp_row0 = row_base + warp * 16;
-  const bool active = warp_row0 < sh.BG;
-  const size_t sh_idx = (size_t)s * sh.Hkv + h;
+  const int num_tiles = max(0, min(ntiles, t_begin + plan.tiles_per_split) - t_begin);
 
-  // queries of this row tile: row r -> (b = r / G, g = r % G), head h*G + g
-  for (int id = tid; id < kRowsPerCta * (D / 8); id += kSelThreads) {
-    const int r = id / (D / 8), c = id % (D / 8);
-    const int row = row_base + r;
-    const bool ok = row < sh.BG;
-    const __nv_bfloat16 *src = a.q;
-    if (ok) {
-      const int b = row / sh.G, g = row % sh.G;
-      src = a.q + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D + c * 8;
-    }
-    cp_async16(smem_addr(sQ) + SwizzledTile<D>::offset(r, c), src, ok);
-  }
-  cp_async_commit();
-
-  auto load_tile = [&](int tile, int stage) {
-    unsigned char *sK = sKV + stage * 2 * kTileBytes;
-    unsigned char *sV = sK + kTileBytes;
-    for (int id = tid; id < kKeyTile * (D / 8); id += kSelThreads) {
-      const int r = id / (D / 8), c = id % (D / 8);
-      const int t = tile * kKeyTile + r;
-      bool ok = t < n;
-      const __nv_bfloat16 *ks = a.k, *vs = a.v;
-      if (ok) {
-        const int lp = t / PAGE, slot = t % PAGE;
-        const long long phys = sh.page_table ? (long long)sh.page_table[(size_t)s * sh.max_pages + lp]
-                                             : (long long)s * sh.max_pages + lp;
-        if (phys < 0 || phys >= sh.n_phys) {
-          ok = false;
-          if (c == 0 && slot == 0) raise_status(a.status, kStatusBadIndex);
-        } else {
-          const size_t off = (((size_t)phys * sh.Hkv + h) * PAGE + slot) * D + c * 8;
-          ks = a.k + off;
-          vs = a.v + off;
+  tc::Engine<D, kSelStages> eng;
+  eng.init(smem_raw, a.status);
+  SelectPolicy<D, PAGE> pol{&sh, &plan, &a, &kmap, &vmap, s, h, n, (n + PAGE - 1) / PAGE,
+                            t_begin, rt * kRowsPerCta, (size_t)s * sh.Hkv + h, sh.sl2};
+  float m, l;
+  const bool alive = eng.template run<PAGE>(pol, num_tiles, m, l);
+  if (eng.warp >= 2) {
+    const int row = rt * kRowsPerCta + eng.row_in_tile();
+    const bool row_ok = row < sh.BG;
+    const size_t prow = ((pol.sh_idx * plan.splits + split) * sh.BG + row);
+    if (alive) {
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        eng.load_o(c0, o);
+        if (row_ok) {
+          float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * D + c0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
-      cp_async16(smem_addr(sK) + SwizzledTile<D>::offset(r, c), ks, ok);
-      cp_async16(smem_addr(sV) + SwizzledTile<D>::offset(r, c), vs, ok);
     }
-    cp_async_commit();
-  };
-
-  WarpAttn<D> wa;
-  wa.init();
-  if (t_begin < t_end) load_tile(t_begin, 0);
-  for (int tile = t_begin; tile < t_end; ++tile) {
-    const int stage = (tile - t_begin) & 1;
-    if (tile + 1 < t_end) {
-      load_tile(tile + 1, stage ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (tile == t_begin && active) wa.load_q(smem_addr(sQ), warp * 16, lane);
-    if (active) {
-      const uint32_t sK = smem_addr(sKV + stage * 2 * kTileBytes);
-      const uint32_t sV = sK + kTileBytes;
-      float acc[WarpAttn<D>::kSNTiles][4];
-      wa.scores(sK, acc, lane);
-      const int t0 = tile * kKeyTile;
-      float page_sum[kKeyTile / PAGE][2];
-      float m_new[2];
-      wa.template softmax_update<PAGE>(acc, sh.sl2, [&](int col) { return t0 + col < n; }, lane,
-                                       page_sum, m_new);
-      if ((lane & 3) == 0) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int row = warp_row0 + (lane >> 2) + 8 * r;
-          if (row < sh.BG) {
-            a.mtile[(sh_idx * plan.max_tiles + tile) * sh.BG + row] = m_new[r];
-#pragma unroll
-            for (int pi = 0; pi < kKeyTile / PAGE; ++pi) {
-              const int lp = t0 / PAGE + pi;
-              if (lp < np) a.pagepart[(sh_idx * sh.max_pages + lp) * sh.BG + row] = page_sum[pi][r];
-            }
-          }
-        }
-      }
-      wa.pv(sV, acc, lane);
-    }
-    __syncthreads();
+    if (row_ok)
+      *reinterpret_cast<float2 *>(a.part_ml + prow * 2) =
+          alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
   }
-  if (t_begin >= t_end) cp_async_wait<0>();
-
-  // split partials (unnormalised O, m, l) of the warp's rows
-  if (active) {
-    const size_t base = (sh_idx * plan.splits + split) * sh.BG;
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int row = warp_row0 + (lane >> 2) + 8 * r;
-      if (row >= sh.BG) continue;
-      float *dst = a.part_o + (base + row) * D;
-#pragma unroll
-      for (int i = 0; i < WarpAttn<D>::kONTiles; ++i) {
-        const int col = i * 8 + 2 * (lane & 3);
-        *reinterpret_cast<float2 *>(dst + col) = make_float2(wa.o[i][2 * r], wa.o[i][2 * r + 1]);
-      }
-      if ((lane & 3) == 0)
-        *reinterpret_cast<float2 *>(a.part_ml + (base + row) * 2) = make_float2(wa.m[r], wa.l[r]);
-    }
-  }
+  eng.teardown();
 }
 
 constexpr int kFinThreads = 256;
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(kFinThreads) select_finalize(const PartialPara
       if (lp >= sh.max_pages) break;
       float acc = 0.f;
       if (lp < np) {
-        const int tile = lp * PAGE / kKeyTile;
+        const int tile = lp * PAGE / tc::kBN;
         const float *part = a.pagepart + (sh_idx * sh.max_pages + lp) * sh.BG;
         const float *mt = a.mtile + (sh_idx * plan.max_tiles + tile) * sh.BG;
         for (int row = lane; row < sh.BG; row += 32)
@@ -358,12 +363,18 @@ template <int D, int PAGE>
 cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectArgs &a,
                          cudaStream_t stream) {
   PartialParams pp{sh, plan, a};
-  const size_t smem = (size_t)kRowsPerCta * D * 2 + 2 * 2 * (size_t)kKeyTile * D * 2;
-  auto kern = select_partial<D, PAGE>;
-  cudaError_t err = set_smem_once(kern, smem);
+  CUtensorMap kmap, vmap;
+  const long long rows = sh.n_phys * sh.Hkv * PAGE;
+  cudaError_t err = make_kv_tensor_map(&kmap, a.k, rows, D, PAGE);
+  if (err != cudaSuccess) return err;
+  err = make_kv_tensor_map(&vmap, a.v, rows, D, PAGE);
+  if (err != cudaSuccess) return err;
+  constexpr auto kern = select_partial<D, PAGE>;
+  constexpr size_t smem = tc::Layout<D, kSelStages>::kAlloc;
+  err = set_smem_once<kern>(smem);
   if (err != cudaSuccess) return err;
   dim3 grid(plan.splits * plan.rowtiles, sh.Hkv, sh.S);
-  kern<<<grid, kSelThreads, smem, stream>>>(pp);
+  kern<<<grid, tc::kThreads, smem, stream>>>(pp, kmap, vmap);
   const int score_ctas = (sh.max_pages + kPagesPerFinCta - 1) / kPagesPerFinCta;
   const int o_ctas = (sh.BG + kRowsPerFinCta - 1) / kRowsPerFinCta;
   select_finalize<D, PAGE><<<dim3(score_ctas + o_ctas, sh.Hkv, sh.S), kFinThreads, 0, stream>>>(pp);
@@ -376,9 +387,9 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
 SelectPlan plan_select(const Shape &sh, int num_sms) {
   SelectPlan p{};
   p.rowtiles = (sh.BG + kRowsPerCta - 1) / kRowsPerCta;
-  p.max_tiles = (int)(((long long)sh.max_pages * sh.P + kKeyTile - 1) / kKeyTile);
+  p.max_tiles = (int)(((long long)sh.max_pages * sh.P + tc::kBN - 1) / tc::kBN);
   const long long base = (long long)sh.S * sh.Hkv * p.rowtiles;
-  const long long target = 2LL * num_sms;  // two resident CTAs per SM
+  const long long target = num_sms;  // one resident CTA per SM
   int splits = (int)std::max(1LL, (target + base - 1) / base);
   splits = std::min(splits, p.max_tiles);
   p.tiles_per_split = (p.max_tiles + splits - 1) / splits;

@@ -4,22 +4,24 @@
 // to the tokens of the selected pages of its KV head plus the block's own B
 // tokens, with no mask inside the block.
 //
-// Two launches on the caller's stream:
-//   1. sparse_partial: CTA = (64-key tile, row tile) x KV head x sequence.  The
-//      key list of a (seq, KV head) is its selected pages in idx order followed by
-//      the block's own tokens; tile t covers keys [64t, 64t+64).  The CTA gathers
-//      its keys/values (page table lookup, bounds-checked), runs 8 warps x 16 rows
-//      of attention and writes an unnormalised partial (O, m, l).
-//   2. sparse_merge: one warp per query row merges the tiles' partials into o_out.
+// One launch per step.  A thread-block cluster of C CTAs serves one (sequence,
+// KV head, 128-row tile): CTA c runs the tcgen05 engine (tc_attn.cuh) over its
+// slice [c*ppc, (c+1)*ppc) of the selected pages, gathered page by page with TMA
+// through the page table; the last CTA also takes the block's own tokens
+// (a 3-D TMA box over blk_k / blk_v).  The C partial results (unnormalised O in
+// shared memory, row max m and sum l) are merged through distributed shared
+// memory: after a cluster barrier CTA c reads every CTA's (m, l, O) for its
+// share of the rows and writes those rows of o_out in bf16.
 #include <algorithm>
 
-#include "attn_core.cuh"
 #include "launch.h"
+#include "sm100.cuh"
+#include "tc_attn.cuh"
 
 namespace dsa {
 namespace {
 
-constexpr int kSpThreads = 256;
+constexpr int kSpStages = 2;
 constexpr int kRowsPerCta = 128;
 
 struct SparseParams {
@@ -29,175 +31,283 @@ struct SparseParams {
 };
 
 template <int D, int PAGE>
-__global__ void __launch_bounds__(kSpThreads, 2) sparse_partial(const SparseParams prm) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ unsigned char key_ok[kKeyTile];
-  const Shape &sh = prm.sh;
-  const SparsePlan &plan = prm.plan;
-  const SparseArgs &a = prm.a;
-  constexpr int kTileBytes = kKeyTile * D * 2;
-  constexpr int kPagesPerTile = kKeyTile / PAGE;
-  unsigned char *sQ = smem;
-  unsigned char *sK = smem + kRowsPerCta * D * 2;
-  unsigned char *sV = sK + kTileBytes;
+struct SparsePolicy {
+  static constexpr int kPagesPerTile = tc::kBN / PAGE;
+  const Shape *sh;
+  const SparseArgs *a;
+  const CUtensorMap *kmap, *vmap, *bkmap, *bvmap;
+  int s, h, n, np, e_begin, e_end, sel_tiles, row_base;
+  size_t sh_idx;
+  float sl2;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int s = blockIdx.z, h = blockIdx.y;
-  const int tile = blockIdx.x / plan.rowtiles, rt = blockIdx.x % plan.rowtiles;
-  const size_t sh_idx = (size_t)s * sh.Hkv + h;
-  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status,
-                             tid == 0 && blockIdx.x == 0 && h == 0);
-  const int np = (n + PAGE - 1) / PAGE;
-  int cnt = a.idx_cnt[sh_idx];
-  if (cnt < 0 || cnt > sh.kmax) {
-    if (tid == 0 && tile == 0 && rt == 0) raise_status(a.status, kStatusBadIndex);
-    cnt = max(0, min(cnt, sh.kmax));
+  // physical page of selected entry e, or -1 if the entry is not usable
+  __device__ __forceinline__ long long phys_of(int e, int &lp) const {
+    lp = -1;
+    if (e >= e_end) return -1;
+    lp = a->idx[sh_idx * sh->kmax + e];
+    if (lp < 0 || lp >= np) return -1;
+    const long long p = sh->page_table ? (long long)sh->page_table[(size_t)s * sh->max_pages + lp]
+                                       : (long long)s * sh->max_pages + lp;
+    return (p >= 0 && p < sh->n_phys) ? p : -1;
   }
-  const int sel_tiles = (cnt * PAGE + kKeyTile - 1) / kKeyTile;
-  const int row_base = rt * kRowsPerCta;
-  const int warp_row0 = row_base + warp * 16;
-  const bool active = warp_row0 < sh.BG;
-  const size_t base = (sh_idx * plan.ntiles + tile) * sh.BG;
-
-  const bool is_sel = tile < sel_tiles;
-  const int btile = tile - sel_tiles;
-  const bool is_blk = !is_sel && btile < plan.blk_tiles;
-  if (!is_sel && !is_blk) {  // past this head's keys: an empty partial
-    for (int row = row_base + tid; row < min(sh.BG, row_base + kRowsPerCta); row += kSpThreads)
-      *reinterpret_cast<float2 *>(a.part_ml + (base + row) * 2) = make_float2(-INFINITY, 0.f);
-    return;
+  __device__ __forceinline__ void prefetch() const {
+    sm100::tma_prefetch_map(kmap);
+    sm100::tma_prefetch_map(vmap);
+    sm100::tma_prefetch_map(bkmap);
+    sm100::tma_prefetch_map(bvmap);
   }
-
-  for (int id = tid; id < kRowsPerCta * (D / 8); id += kSpThreads) {
-    const int r = id / (D / 8), c = id % (D / 8);
-    const int row = row_base + r;
-    const bool ok = row < sh.BG;
-    const __nv_bfloat16 *src = a.q;
-    if (ok) {
-      const int b = row / sh.G, g = row % sh.G;
-      src = a.q + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D + c * 8;
-    }
-    cp_async16(smem_addr(sQ) + SwizzledTile<D>::offset(r, c), src, ok);
-  }
-  for (int id = tid; id < kKeyTile * (D / 8); id += kSpThreads) {
-    const int r = id / (D / 8), c = id % (D / 8);
-    bool ok;
-    const __nv_bfloat16 *ks = a.k, *vs = a.v;
-    if (is_sel) {
-      const int e = tile * kPagesPerTile + r / PAGE, slot = r % PAGE;
-      ok = e < cnt;
-      if (ok) {
-        const int lp = a.idx[sh_idx * sh.kmax + e];
-        const bool lp_ok = lp >= 0 && lp < np;
-        long long phys = -1;
-        if (lp_ok)
-          phys = sh.page_table ? (long long)sh.page_table[(size_t)s * sh.max_pages + lp]
-                               : (long long)s * sh.max_pages + lp;
-        if (!lp_ok || phys < 0 || phys >= sh.n_phys) {
-          ok = false;
-          if (c == 0 && slot == 0) raise_status(a.status, kStatusBadIndex);
-        } else {
-          ok = lp * PAGE + slot < n;
-          const size_t off = (((size_t)phys * sh.Hkv + h) * PAGE + slot) * D + c * 8;
-          ks = a.k + off;
-          vs = a.v + off;
+  __device__ __forceinline__ void load_tile(int k, uint32_t sk, uint32_t sv, uint32_t half_bytes,
+                                            uint32_t bar) const {
+    if (k < sel_tiles) {
+      const int e0 = e_begin + k * kPagesPerTile;
+      long long phys[kPagesPerTile];
+      uint32_t nvalid = 0;
+#pragma unroll
+      for (int pi = 0; pi < kPagesPerTile; ++pi) {
+        int lp;
+        phys[pi] = phys_of(e0 + pi, lp);
+        if (phys[pi] >= 0) ++nvalid;
+        else if (e0 + pi < e_end) raise_status(a->status, kStatusBadIndex);
+      }
+      sm100::mbar_arrive_expect_tx(bar, nvalid * PAGE * 128u * (D / 64) * 2u);
+#pragma unroll
+      for (int pi = 0; pi < kPagesPerTile; ++pi) {
+        if (phys[pi] < 0) continue;
+        const int y = (int)((phys[pi] * sh->Hkv + h) * PAGE);
+#pragma unroll
+        for (int hf = 0; hf < D / 64; ++hf) {
+          sm100::tma_load_2d(sk + hf * half_bytes + pi * PAGE * 128, kmap, bar, hf * 64, y);
+          sm100::tma_load_2d(sv + hf * half_bytes + pi * PAGE * 128, vmap, bar, hf * 64, y);
         }
       }
-    } else {
-      const int u = btile * kKeyTile + r;
-      ok = u < sh.B;
-      if (ok) {
-        const size_t off = (((size_t)s * sh.B + u) * sh.Hkv + h) * D + c * 8;
-        ks = a.blk_k + off;
-        vs = a.blk_v + off;
+    } else {  // the block's own tokens u = 64j .. 64j+63 of this sequence
+      const int j = k - sel_tiles;
+      sm100::mbar_arrive_expect_tx(bar, 64u * 128u * (D / 64) * 2u);
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        sm100::tma_load_3d(sk + hf * half_bytes, bkmap, bar, hf * 64, h, s * sh->B + j * 64);
+        sm100::tma_load_3d(sv + hf * half_bytes, bvmap, bar, hf * 64, h, s * sh->B + j * 64);
       }
     }
-    if (c == 0) key_ok[r] = ok;
-    cp_async16(smem_addr(sK) + SwizzledTile<D>::offset(r, c), ks, ok);
-    cp_async16(smem_addr(sV) + SwizzledTile<D>::offset(r, c), vs, ok);
   }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-  if (!active) return;
-
-  WarpAttn<D> wa;
-  wa.init();
-  wa.load_q(smem_addr(sQ), warp * 16, lane);
-  float acc[WarpAttn<D>::kSNTiles][4];
-  wa.scores(smem_addr(sK), acc, lane);
-  float m_new[2];
-  wa.template softmax_update<0>(acc, sh.sl2, [&](int col) { return key_ok[col] != 0; }, lane,
-                                nullptr, m_new);
-  wa.pv(smem_addr(sV), acc, lane);
+  __device__ __forceinline__ const __nv_bfloat16 *q_row(int r) const {
+    const int row = row_base + r;
+    if (row >= sh->BG) return nullptr;
+    const int b = row / sh->G, g = row % sh->G;
+    return a->q + (((size_t)s * sh->B + b) * sh->Hq + (size_t)h * sh->G + g) * D;
+  }
+  __device__ __forceinline__ uint64_t key_mask(int k) const {
+    uint64_t m = 0;
+    if (k < sel_tiles) {
+      const int e0 = e_begin + k * kPagesPerTile;
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int row = warp_row0 + (lane >> 2) + 8 * r;
-    if (row >= sh.BG) continue;
-    float *dst = a.part_o + (base + row) * D;
-#pragma unroll
-    for (int i = 0; i < WarpAttn<D>::kONTiles; ++i) {
-      const int col = i * 8 + 2 * (lane & 3);
-      *reinterpret_cast<float2 *>(dst + col) = make_float2(wa.o[i][2 * r], wa.o[i][2 * r + 1]);
+      for (int pi = 0; pi < kPagesPerTile; ++pi) {
+        int lp;
+        if (phys_of(e0 + pi, lp) < 0) continue;
+        const int cnt = min(PAGE, n - lp * PAGE);
+        if (cnt > 0) m |= ((cnt >= 64) ? ~0ull : ((1ull << cnt) - 1ull)) << (pi * PAGE);
+      }
+    } else {
+      const int cnt = min(64, sh->B - (k - sel_tiles) * 64);
+      if (cnt > 0) m = (cnt >= 64) ? ~0ull : ((1ull << cnt) - 1ull);
     }
-    if ((lane & 3) == 0)
-      *reinterpret_cast<float2 *>(a.part_ml + (base + row) * 2) = make_float2(wa.m[r], wa.l[r]);
+    return m;
   }
-}
+  __device__ __forceinline__ void after_tile(int, int, float, const float *) const {}
+};
 
-constexpr int kMergeThreads = 256;
-
-template <int D>
-__global__ void __launch_bounds__(kMergeThreads) sparse_merge(const SparseParams prm) {
+template <int D, int PAGE>
+__global__ void __launch_bounds__(tc::kThreads, 1)
+    sparse_attn(const SparseParams prm, const __grid_constant__ CUtensorMap kmap,
+                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap bkmap,
+                const __grid_constant__ CUtensorMap bvmap) {
+  using L = tc::Layout<D, kSpStages>;
+  extern __shared__ unsigned char smem_raw[];
   const Shape &sh = prm.sh;
   const SparsePlan &plan = prm.plan;
   const SparseArgs &a = prm.a;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int s = blockIdx.z, h = blockIdx.y;
-  const int row = blockIdx.x * (kMergeThreads / 32) + warp;
-  if (row >= sh.BG) return;
+  const int C = plan.cluster;   // cluster size == gridDim.x
+  const int c = blockIdx.x;     // rank in the cluster
+  const int h = blockIdx.y;
+  const int s = blockIdx.z / plan.rowtiles, rt = blockIdx.z % plan.rowtiles;
   const size_t sh_idx = (size_t)s * sh.Hkv + h;
-  float M = -INFINITY;
-  for (int t = lane; t < plan.ntiles; t += 32) {
-    const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + ((sh_idx * plan.ntiles + t) * sh.BG + row) * 2);
-    if (ml.y > 0.f) M = fmaxf(M, ml.x);
+  const bool reporter = threadIdx.x == 0 && c == 0 && rt == 0;
+  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status, reporter && h == 0);
+  int cnt = a.idx_cnt[sh_idx];
+  if (cnt < 0 || cnt > sh.kmax) {
+    if (reporter) raise_status(a.status, kStatusBadIndex);
+    cnt = max(0, min(cnt, sh.kmax));
   }
-  M = warp_max(M);
-  constexpr int kPer = D / 32;
-  float acc[kPer];
+  const int e_begin = min(cnt, c * plan.ppc), e_end = min(cnt, (c + 1) * plan.ppc);
+  constexpr int kPagesPerTile = tc::kBN / PAGE;
+  const int sel_tiles = (e_end - e_begin + kPagesPerTile - 1) / kPagesPerTile;
+  const int num_tiles = sel_tiles + (c == C - 1 ? plan.blk_tiles : 0);
+  const int row_base = rt * kRowsPerCta;
+
+  tc::Engine<D, kSpStages> eng;
+  eng.init(smem_raw, a.status);
+  SparsePolicy<D, PAGE> pol{&sh, &a, &kmap, &vmap, &bkmap, &bvmap, s, h, n,
+                            (n + PAGE - 1) / PAGE, e_begin, e_end, sel_tiles, row_base,
+                            sh_idx, sh.sl2};
+  float m, l;
+  const bool alive = eng.template run<PAGE>(pol, num_tiles, m, l);
+
+  // ---- this CTA's partial into its shared memory (the K/V/P area is free now)
+  constexpr int kOStride = D + 4;  // floats per row, padded against bank conflicts
+  float *obuf = reinterpret_cast<float *>(eng.smem + L::kOffKV);
+  float2 *ml = reinterpret_cast<float2 *>(eng.smem + L::kOffKV + 128 * kOStride * 4);
+  float2 *gml = ml + 128;                                   // [rows][C] gathered (m, l)
+  float *wts = reinterpret_cast<float *>(gml + 128 + 16);   // [rows][C] merge weights
+  static_assert(L::kOffKV + 128 * kOStride * 4 + (128 + 128 + 16) * 8 + (128 + 16) * 4 <= L::kOffBar,
+                "merge buffers must fit in the K/V/P area");
+  if (eng.warp >= 2) {
+    const int r = eng.row_in_tile();
+    if (alive) {
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
-  float L = 0.f;
-  for (int t = 0; t < plan.ntiles; ++t) {
-    const size_t r = (sh_idx * plan.ntiles + t) * sh.BG + row;
-    const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + r * 2);
-    if (!(ml.y > 0.f)) continue;
-    const float w = exp2f(ml.x - M);
-    L += w * ml.y;
-    const float *src = a.part_o + r * D + lane * kPer;
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        eng.load_o(c0, o);
+        float4 *dst = reinterpret_cast<float4 *>(obuf + r * kOStride + c0);
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) acc[i] += w * src[i];
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                               __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+      }
+    }
+    ml[r] = alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
   }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  const int b = row / sh.G, g = row % sh.G;
-  __nv_bfloat16 *dst = a.o_out + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D + lane * kPer;
-#pragma unroll
-  for (int i = 0; i < kPer; i += 2)
-    *reinterpret_cast<__nv_bfloat162 *>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+  sm100::cluster_sync();
+
+  // ---- merge: CTA c owns rows [c*rpc, (c+1)*rpc) of the tile
+  const int rows_here = min(kRowsPerCta, sh.BG - row_base);
+  const int rpc = (kRowsPerCta + C - 1) / C;
+  const int r0 = c * rpc;
+  const int r1 = min(rows_here, r0 + rpc);
+  const int nrows = max(0, r1 - r0);
+  const uint32_t ml_addr = smem_addr(ml), o_addr = smem_addr(obuf);
+  for (int t = threadIdx.x; t < nrows * C; t += blockDim.x) {
+    const int rl = t / C, j = t % C;
+    gml[t] = sm100::ld_cluster_f2(sm100::cluster_map(ml_addr + (r0 + rl) * 8, j));
+  }
+  __syncthreads();
+  for (int rl = threadIdx.x; rl < nrows; rl += blockDim.x) {
+    float M = -INFINITY;
+    for (int j = 0; j < C; ++j)
+      if (gml[rl * C + j].y > 0.f) M = fmaxf(M, gml[rl * C + j].x);
+    float Lsum = 0.f;
+    for (int j = 0; j < C; ++j) {
+      const float2 v = gml[rl * C + j];
+      const float w = v.y > 0.f ? exp2f(v.x - M) : 0.f;
+      wts[rl * C + j] = w;
+      Lsum += w * v.y;
+    }
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    for (int j = 0; j < C; ++j) wts[rl * C + j] *= inv;
+  }
+  __syncthreads();
+  constexpr int kQuads = D / 4;
+  for (int t = threadIdx.x; t < nrows * kQuads; t += blockDim.x) {
+    const int rl = t / kQuads, q4 = t % kQuads;
+    const int row = r0 + rl;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < C; ++j) {
+      const float w = wts[rl * C + j];
+      if (w == 0.f) continue;  // an empty partial: its buffer holds no data
+      const float4 v =
+          sm100::ld_cluster_f4(sm100::cluster_map(o_addr + (row * kOStride + 4 * q4) * 4, j));
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
+    }
+    const int grow = row_base + row;
+    const int b = grow / sh.G, g = grow % sh.G;
+    __nv_bfloat16 *dst =
+        a.o_out + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D + 4 * q4;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<uint32_t *>(&lo);
+    packed.y = *reinterpret_cast<uint32_t *>(&hi);
+    *reinterpret_cast<uint2 *>(dst) = packed;
+  }
+  sm100::cluster_sync();  // no CTA leaves while another may still read its shared memory
+  eng.teardown();
+}
+
+// Largest cluster size (16, 8, 4, 2) that the device can schedule with this
+// kernel's shared memory, queried once per device; 1 if none.
+template <auto K>
+int max_cluster(size_t smem) {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int best = 1;
+    for (int cs = 16; cs >= 2; cs >>= 1) {
+      if (cs > 8 &&
+          cudaFuncSetAttribute(K, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cs, 1, 1);
+      cfg.blockDim = dim3(tc::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cs;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int nclusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&nclusters, K, &cfg) == cudaSuccess && nclusters >= 1) {
+        best = cs;
+        break;
+      }
+      cudaGetLastError();
+    }
+    cached[dev] = best;
+  }
+  return cached[dev];
 }
 
 template <int D, int PAGE>
-cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan, const SparseArgs &a,
+cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan_in, const SparseArgs &a,
                          cudaStream_t stream) {
-  SparseParams prm{sh, plan, a};
-  const size_t smem = (size_t)kRowsPerCta * D * 2 + 2 * (size_t)kKeyTile * D * 2;
-  auto kern = sparse_partial<D, PAGE>;
-  cudaError_t err = set_smem_once(kern, smem);
+  constexpr auto kern = sparse_attn<D, PAGE>;
+  constexpr size_t smem = tc::Layout<D, kSpStages>::kAlloc;
+  cudaError_t err = set_smem_once<kern>(smem);
   if (err != cudaSuccess) return err;
-  kern<<<dim3(plan.ntiles * plan.rowtiles, sh.Hkv, sh.S), kSpThreads, smem, stream>>>(prm);
-  const int rows_per_cta = kMergeThreads / 32;
-  sparse_merge<D><<<dim3((sh.BG + rows_per_cta - 1) / rows_per_cta, sh.Hkv, sh.S), kMergeThreads, 0,
-                    stream>>>(prm);
+  SparsePlan plan = plan_in;
+  const int cap = max_cluster<kern>(smem);
+  if (plan.cluster > cap) {
+    plan.cluster = cap;
+    plan.ppc = (sh.kmax + cap - 1) / cap;
+  }
+  CUtensorMap kmap, vmap, bkmap, bvmap;
+  const long long rows = sh.n_phys * sh.Hkv * PAGE;
+  if ((err = make_kv_tensor_map(&kmap, a.k, rows, D, PAGE)) != cudaSuccess) return err;
+  if ((err = make_kv_tensor_map(&vmap, a.v, rows, D, PAGE)) != cudaSuccess) return err;
+  if ((err = make_blk_tensor_map(&bkmap, a.blk_k, (long long)sh.S * sh.B, sh.Hkv, D)) != cudaSuccess)
+    return err;
+  if ((err = make_blk_tensor_map(&bvmap, a.blk_v, (long long)sh.S * sh.B, sh.Hkv, D)) != cudaSuccess)
+    return err;
+  SparseParams prm{sh, plan, a};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.cluster, sh.Hkv, sh.S * plan.rowtiles);
+  cfg.blockDim = dim3(tc::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = plan.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, prm, kmap, vmap, bkmap, bvmap);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
@@ -206,15 +316,12 @@ cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan, const SparseAr
 SparsePlan plan_sparse(const Shape &sh, int /*num_sms*/) {
   SparsePlan p{};
   p.rowtiles = (sh.BG + kRowsPerCta - 1) / kRowsPerCta;
-  p.sel_tiles = (int)(((long long)sh.kmax * sh.P + kKeyTile - 1) / kKeyTile);
-  p.blk_tiles = (sh.B + kKeyTile - 1) / kKeyTile;
-  p.ntiles = p.sel_tiles + p.blk_tiles;
-  auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
-  size_t off = 4096;
-  const size_t shn = (size_t)sh.S * sh.Hkv;
-  p.off_part_o = off;  off = align(off + shn * p.ntiles * sh.BG * sh.d * 4);
-  p.off_part_ml = off; off = align(off + shn * p.ntiles * sh.BG * 2 * 4);
-  p.total = off;
+  int cs = std::min(16, std::max(1, sh.kmax));
+  while (cs & (cs - 1)) cs &= cs - 1;  // power of two
+  p.cluster = cs;
+  p.ppc = (sh.kmax + cs - 1) / cs;
+  p.blk_tiles = (sh.B + tc::kBN - 1) / tc::kBN;
+  p.total = 4096;  // status word only: partials never leave the cluster
   return p;
 }
 
