@@ -84,7 +84,7 @@ def test_workspace_too_small_rejected(lib):
     dims = good_dims()
     ok = ctypes.c_void_p(1 << 20)
     need = lib.dsa_sparse_workspace_size(ctypes.byref(dims))
-    assert need > 4096
+    assert need >= 4096  # at least the status header
     rc = lib.dsa_sparse_attn(ok, ok, ok, ok, ok, ok, ok, None, ctypes.byref(dims), ok, ok, ok,
                              need - 1)
     assert rc == dsa.DSA_ERR_WORKSPACE_TOO_SMALL
