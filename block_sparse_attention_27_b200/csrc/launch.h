@@ -22,6 +22,11 @@ struct Shape {
 cudaError_t make_kv_tensor_map(CUtensorMap *out, const void *base, long long rows, int D,
                                int box_rows);
 
+// The same cache as 4-D (D, P, Hkv, n_phys); boxes of 64 elements x P tokens x 1 head
+// x `pages` consecutive physical pages (tmap.cu).
+cudaError_t make_kv_pages_tensor_map(CUtensorMap *out, const void *base, long long n_phys, int Hkv,
+                                     int P, int D, int pages);
+
 // The block's own keys/values [S*B, Hkv, D] bf16; boxes of 64 elements x 1 head x
 // 64 tokens with the 128-byte swizzle (tmap.cu).
 cudaError_t make_blk_tensor_map(CUtensorMap *out, const void *base, long long tokens, int Hkv,
@@ -37,6 +42,7 @@ struct SelectPlan {
   int splits;           // key splits per (seq, KV head, row tile)
   int tiles_per_split;  // 64-token tiles per split
   int max_tiles;        // ceil(max_pages * P / 64)
+  int fin_pages;        // pages per score CTA of the finalize pass
   size_t off_part_o, off_part_ml, off_pagepart, off_mtile, off_scores, total;
 };
 

@@ -39,27 +39,35 @@ struct PartialParams {
 // and that max (mtile); the split's unnormalised O row, m and l go to part_o /
 // part_ml.
 // ---------------------------------------------------------------------------
-constexpr int kSelStages = 4;
+constexpr int kSelStages = 5;
 
 template <int D, int PAGE>
 struct SelectPolicy {
-  const Shape *sh;
-  const SelectPlan *plan;
-  const SelectArgs *a;
-  const CUtensorMap *kmap, *vmap;
-  int s, h, n, np, t_begin, row_base;
-  size_t sh_idx;
+  // everything the hot loops touch is held by value (registers), with base
+  // pointers already offset to this (sequence, KV head)
+  static constexpr bool kIssueBeforeSync = true;  // tile addresses need no table
+  const CUtensorMap *kmap, *vmap;    // one page per box
+  const CUtensorMap *kmap4, *vmap4;  // 64/PAGE consecutive pages per box
+  const int32_t *page_row;          // page-table row of the sequence, or null (identity)
+  const __nv_bfloat16 *q_head;      // q[s, 0, h*G, 0]
+  float *mtile_head;                // mtile[s, h, 0, 0]
+  float *pagepart_head;             // pagepart[s, h, 0, 0]
+  uint32_t *status;
+  long long n_phys, phys0;          // phys0 = s*max_pages (identity map)
+  int Hkv, h, G, Hq, BG, n, np, t_begin, row_base;
   float sl2;
 
   __device__ __forceinline__ long long phys_of(int lp) const {
     if (lp >= np) return -1;
-    const long long p = sh->page_table ? (long long)sh->page_table[(size_t)s * sh->max_pages + lp]
-                                       : (long long)s * sh->max_pages + lp;
-    return (p >= 0 && p < sh->n_phys) ? p : -1;
+    const long long p = page_row ? (long long)page_row[lp] : phys0 + lp;
+    return (p >= 0 && p < n_phys) ? p : -1;
   }
+  __device__ __forceinline__ void prepare(unsigned char *) const {}
   __device__ __forceinline__ void prefetch() const {
     sm100::tma_prefetch_map(kmap);
     sm100::tma_prefetch_map(vmap);
+    sm100::tma_prefetch_map(kmap4);
+    sm100::tma_prefetch_map(vmap4);
   }
   __device__ __forceinline__ void load_tile(int k, uint32_t sk, uint32_t sv, uint32_t half_bytes,
                                             uint32_t bar) const {
@@ -67,17 +75,27 @@ struct SelectPolicy {
     const int lp0 = (t_begin + k) * tc::kBN / PAGE;
     long long phys[kPages];
     uint32_t nvalid = 0;
+    bool run = true;  // all pages valid and physically consecutive
 #pragma unroll
     for (int pi = 0; pi < kPages; ++pi) {
       phys[pi] = phys_of(lp0 + pi);
       if (phys[pi] >= 0) ++nvalid;
-      else if (lp0 + pi < np && blockIdx.x == 0) raise_status(a->status, kStatusBadIndex);
+      else if (lp0 + pi < np && blockIdx.x == 0) raise_status(status, kStatusBadIndex);
+      run = run && phys[pi] >= 0 && phys[pi] == phys[0] + pi;
     }
     sm100::mbar_arrive_expect_tx(bar, nvalid * PAGE * 128u * (D / 64) * 2u);
+    if (kPages > 1 && run) {  // the whole tile in one box per half
+#pragma unroll
+      for (int hf = 0; hf < D / 64; ++hf) {
+        sm100::tma_load_4d(sk + hf * half_bytes, kmap4, bar, hf * 64, 0, h, (int)phys[0]);
+        sm100::tma_load_4d(sv + hf * half_bytes, vmap4, bar, hf * 64, 0, h, (int)phys[0]);
+      }
+      return;
+    }
 #pragma unroll
     for (int pi = 0; pi < kPages; ++pi) {
       if (phys[pi] < 0) continue;
-      const int y = (int)((phys[pi] * sh->Hkv + h) * PAGE);
+      const int y = (int)((phys[pi] * Hkv + h) * PAGE);
 #pragma unroll
       for (int hf = 0; hf < D / 64; ++hf) {
         sm100::tma_load_2d(sk + hf * half_bytes + pi * PAGE * 128, kmap, bar, hf * 64, y);
@@ -87,12 +105,14 @@ struct SelectPolicy {
   }
   __device__ __forceinline__ const __nv_bfloat16 *q_row(int r) const {
     const int row = row_base + r;
-    if (row >= sh->BG) return nullptr;
-    const int b = row / sh->G, g = row % sh->G;
-    return a->q + (((size_t)s * sh->B + b) * sh->Hq + (size_t)h * sh->G + g) * D;
+    if (row >= BG) return nullptr;
+    const int b = row / G, g = row % G;
+    return q_head + ((size_t)b * Hq + g) * D;
   }
   __device__ __forceinline__ uint64_t key_mask(int k) const {
     const int t0 = (t_begin + k) * tc::kBN;
+    if (t0 + tc::kBN <= n && !page_row && phys0 + (t0 + tc::kBN - 1) / PAGE < n_phys)
+      return ~0ull;  // a full tile of pages that are all in the cache
     uint64_t m = 0;
 #pragma unroll
     for (int pi = 0; pi < tc::kBN / PAGE; ++pi) {
@@ -103,23 +123,29 @@ struct SelectPolicy {
     }
     return m;
   }
-  __device__ __forceinline__ void after_tile(int k, int r, float m_used, const float *psum) const {
+  // per-unit masses of tile k (a unit is min(PAGE, 32) keys of one page),
+  // relative to the row's reference max m_used of the group that ran the tile
+  __device__ __forceinline__ void after_tile(int k, int r, float m_used, const float *usum) const {
+    using U = tc::Units<PAGE>;
     const int row = row_base + r;
-    if (row >= sh->BG) return;
+    if (row >= BG) return;
     const int tile = t_begin + k;
-    a->mtile[(sh_idx * plan->max_tiles + tile) * sh->BG + row] = m_used;
+    mtile_head[(size_t)tile * BG + row] = m_used;
 #pragma unroll
-    for (int pi = 0; pi < tc::kBN / PAGE; ++pi) {
-      const int lp = tile * tc::kBN / PAGE + pi;
-      if (lp < np) a->pagepart[(sh_idx * sh->max_pages + lp) * sh->BG + row] = psum[pi];
+    for (int u = 0; u < U::kPerTile; ++u) {
+      const int t = tile * tc::kBN + u * U::kKeys;
+      const int lp = t / PAGE;
+      if (lp < np)
+        pagepart_head[((size_t)lp * U::kPerPage + (t % PAGE) / U::kKeys) * BG + row] = usum[u];
     }
   }
 };
 
 template <int D, int PAGE>
 __global__ void __launch_bounds__(tc::kThreads, 1)
-    select_partial(const PartialParams pp, const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap) {
+    select_partial(const __grid_constant__ PartialParams pp, const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kmap4,
+                   const __grid_constant__ CUtensorMap vmap4) {
   extern __shared__ unsigned char smem_raw[];
   const Shape &sh = pp.sh;
   const SelectPlan &plan = pp.plan;
@@ -132,56 +158,97 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const int t_begin = split * plan.tiles_per_split;
   const int num_tiles = max(0, min(ntiles, t_begin + plan.tiles_per_split) - t_begin);
 
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
+  const size_t sh_idx = (size_t)s * sh.Hkv + h;
+  SelectPolicy<D, PAGE> pol;
+  pol.kmap = &kmap;
+  pol.vmap = &vmap;
+  pol.kmap4 = &kmap4;
+  pol.vmap4 = &vmap4;
+  pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
+  pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
+  pol.mtile_head = a.mtile + sh_idx * plan.max_tiles * sh.BG;
+  pol.pagepart_head = a.pagepart + sh_idx * sh.max_pages * tc::Units<PAGE>::kPerPage * sh.BG;
+  pol.status = a.status;
+  pol.n_phys = sh.n_phys;
+  pol.phys0 = (long long)s * sh.max_pages;
+  pol.Hkv = sh.Hkv;
+  pol.h = h;
+  pol.G = sh.G;
+  pol.Hq = sh.Hq;
+  pol.BG = sh.BG;
+  pol.n = n;
+  pol.np = (n + PAGE - 1) / PAGE;
+  pol.t_begin = t_begin;
+  pol.row_base = rt * kRowsPerCta;
+  pol.sl2 = sh.sl2;
   tc::Engine<D, kSelStages> eng;
-  eng.init(smem_raw, a.status);
-  SelectPolicy<D, PAGE> pol{&sh, &plan, &a, &kmap, &vmap, s, h, n, (n + PAGE - 1) / PAGE,
-                            t_begin, rt * kRowsPerCta, (size_t)s * sh.Hkv + h, sh.sl2};
+  eng.init(smem_raw, a.status, pol, num_tiles);
   float m, l;
-  const bool alive = eng.template run<PAGE>(pol, num_tiles, m, l);
+  eng.template run<PAGE>(pol, num_tiles, m, l);
+  float m_row, l_row, wa, wb;
+  eng.finish(m, l, m_row, l_row, wa, wb);
   if (eng.warp >= 2) {
+    // O = wa * O_0 + wb * O_1 relative to m_row; this thread writes its half of the columns
+    const int g = eng.group();
     const int row = rt * kRowsPerCta + eng.row_in_tile();
     const bool row_ok = row < sh.BG;
-    const size_t prow = ((pol.sh_idx * plan.splits + split) * sh.BG + row);
-    if (alive) {
+    const size_t prow = ((sh_idx * plan.splits + split) * sh.BG + row);
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        eng.load_o(c0, o);
-        if (row_ok) {
-          float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * D + c0);
+    for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 32) {
+      uint32_t oa[32], ob[32];
+      eng.load_o(0, c0, oa);
+      eng.load_o(1, c0, ob);
+      if (row_ok && l_row > 0.f) {
+        float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * D + c0);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+        for (int i = 0; i < 8; ++i) {
+          float v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = wa > 0.f ? wa * __uint_as_float(oa[4 * i + e]) : 0.f;
+            const float x1 = wb > 0.f ? wb * __uint_as_float(ob[4 * i + e]) : 0.f;
+            v[e] = x0 + x1;
+          }
+          dst[i] = make_float4(v[0], v[1], v[2], v[3]);
         }
       }
     }
-    if (row_ok)
+    if (row_ok && g == 0)
       *reinterpret_cast<float2 *>(a.part_ml + prow * 2) =
-          alive ? make_float2(m, l) : make_float2(-INFINITY, 0.f);
+          l_row > 0.f ? make_float2(m_row, l_row) : make_float2(-INFINITY, 0.f);
+    if (row == rt * kRowsPerCta) DSA_TRACE_EVENT(7);
   }
   eng.teardown();
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(11);
 }
 
+// ---------------------------------------------------------------------------
+// select_finalize: merges the splits.  Every CTA first forms, for each query
+// row, the global reference M = max_j m_j and 1/L with L = sum_j l_j 2^(m_j - M)
+// (one online pass over the splits).  Score CTAs then turn the partial masses of
+// their pages into  S_h[q] = (1/BG) sum_rows pagepart * 2^(mtile - M) / L;
+// output CTAs write o_out = sum_j 2^(m_j - M) O_j / L in bf16.
+// ---------------------------------------------------------------------------
 constexpr int kFinThreads = 256;
-constexpr int kPagesPerFinCta = 64;
 constexpr int kRowsPerFinCta = 8;
 
-// Row max M and 1/L over the splits, into shared memory.
-__device__ void merged_row_stats(const Shape &sh, const SelectPlan &plan, const float *part_ml,
-                                 size_t sh_idx, float *sM, float *sLinv) {
+__device__ __forceinline__ void merged_row_stats(const Shape &sh, const SelectPlan &plan,
+                                                 const float *part_ml, size_t sh_idx, float *sM,
+                                                 float *sLinv) {
   for (int row = threadIdx.x; row < sh.BG; row += blockDim.x) {
-    float M = -INFINITY;
+    float M = -INFINITY, L = 0.f;
+#pragma unroll 4
     for (int j = 0; j < plan.splits; ++j) {
       const float2 ml = *reinterpret_cast<const float2 *>(
           part_ml + ((sh_idx * plan.splits + j) * sh.BG + row) * 2);
-      if (ml.y > 0.f) M = fmaxf(M, ml.x);
-    }
-    float L = 0.f;
-    for (int j = 0; j < plan.splits; ++j) {
-      const float2 ml = *reinterpret_cast<const float2 *>(
-          part_ml + ((sh_idx * plan.splits + j) * sh.BG + row) * 2);
-      if (ml.y > 0.f) L += ml.y * exp2f(ml.x - M);
+      if (!(ml.y > 0.f)) continue;
+      if (ml.x > M) {
+        L = L * exp2f(M - ml.x) + ml.y;
+        M = ml.x;
+      } else {
+        L += ml.y * exp2f(ml.x - M);
+      }
     }
     sM[row] = M;
     sLinv[row] = L > 0.f ? 1.f / L : 0.f;
@@ -189,7 +256,7 @@ __device__ void merged_row_stats(const Shape &sh, const SelectPlan &plan, const 
 }
 
 template <int D, int PAGE>
-__global__ void __launch_bounds__(kFinThreads) select_finalize(const PartialParams pp) {
+__global__ void __launch_bounds__(kFinThreads) select_finalize(const __grid_constant__ PartialParams pp) {
   __shared__ float sM[256], sLinv[256];
   const Shape &sh = pp.sh;
   const SelectPlan &plan = pp.plan;
@@ -201,22 +268,40 @@ __global__ void __launch_bounds__(kFinThreads) select_finalize(const PartialPara
   merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int score_ctas = (sh.max_pages + kPagesPerFinCta - 1) / kPagesPerFinCta;
+  const int score_ctas = (sh.max_pages + plan.fin_pages - 1) / plan.fin_pages;
   if ((int)blockIdx.x < score_ctas) {
+    // a warp takes one 64-token tile (64/PAGE pages) at a time: the row factor
+    // 2^(mtile - M) / L is shared by the tile's pages, and all loads of the tile
+    // are in flight together before the per-page warp reductions
+    using U = tc::Units<PAGE>;
+    constexpr int kPagesPerTile = tc::kBN / PAGE;
+    constexpr int kUnitsPerTile = tc::kBN / U::kKeys;
     const float inv_bg = 1.f / (float)sh.BG;
-    for (int k = warp; k < kPagesPerFinCta; k += kFinThreads / 32) {
-      const int lp = blockIdx.x * kPagesPerFinCta + k;
-      if (lp >= sh.max_pages) break;
-      float acc = 0.f;
-      if (lp < np) {
-        const int tile = lp * PAGE / tc::kBN;
-        const float *part = a.pagepart + (sh_idx * sh.max_pages + lp) * sh.BG;
+    const int p0 = blockIdx.x * plan.fin_pages;  // a multiple of 64 tokens
+    const int p1 = min(sh.max_pages, p0 + plan.fin_pages);
+    for (int lp0 = p0 + warp * kPagesPerTile; lp0 < p1; lp0 += (kFinThreads / 32) * kPagesPerTile) {
+      const int tile = lp0 * PAGE / tc::kBN;
+      float acc[kUnitsPerTile];
+#pragma unroll
+      for (int u = 0; u < kUnitsPerTile; ++u) acc[u] = 0.f;
+      if (lp0 < np) {
         const float *mt = a.mtile + (sh_idx * plan.max_tiles + tile) * sh.BG;
-        for (int row = lane; row < sh.BG; row += 32)
-          acc += part[row] * exp2f(mt[row] - sM[row]) * sLinv[row];
-        acc = warp_sum(acc) * inv_bg;
+        const float *part = a.pagepart + (sh_idx * sh.max_pages + lp0) * U::kPerPage * sh.BG;
+        for (int row = lane; row < sh.BG; row += 32) {
+          const float f = exp2f(mt[row] - sM[row]) * sLinv[row];
+#pragma unroll
+          for (int u = 0; u < kUnitsPerTile; ++u)
+            if (lp0 + u / U::kPerPage < np) acc[u] += part[(size_t)u * sh.BG + row] * f;
+        }
       }
-      if (lane == 0) a.scores[sh_idx * sh.max_pages + lp] = acc;
+#pragma unroll
+      for (int pi = 0; pi < kPagesPerTile; ++pi) {
+        float v = 0.f;
+#pragma unroll
+        for (int u = pi * U::kPerPage; u < (pi + 1) * U::kPerPage; ++u) v += acc[u];
+        v = warp_sum(v) * inv_bg;
+        if (lane == 0 && lp0 + pi < p1) a.scores[sh_idx * sh.max_pages + lp0 + pi] = v;
+      }
     }
   } else {
     const int row = (blockIdx.x - score_ctas) * kRowsPerFinCta + warp;
@@ -243,17 +328,26 @@ __global__ void __launch_bounds__(kFinThreads) select_finalize(const PartialPara
   }
 }
 
+// ---------------------------------------------------------------------------
+// select_topk: one CTA per (sequence, KV head).  Page scores are >= 0, so their
+// fp32 bit patterns order like the values; a 4-pass radix select (8 bits per
+// pass, histogram in shared memory, bin search by one warp) finds the kp-th
+// largest key T.  Pages with key > T are kept, and among keys == T the lowest
+// page indices, so ties go to the lower index; an ordered compaction writes the
+// kept pages in ascending order.
+// ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
+constexpr int kTopkSmemKeys = 11264;  // keys staged in shared memory up to this many pages (44 KB)
 
-// Order-preserving key of a non-negative score (-0 folded onto +0).
 __device__ __forceinline__ uint32_t score_key(float v) {
-  return v > 0.f ? __float_as_uint(v) : 0u;
+  return v > 0.f ? __float_as_uint(v) : 0u;  // -0 folds onto +0
 }
 
-__global__ void __launch_bounds__(kTopkThreads) select_topk(const PartialParams pp) {
+__global__ void __launch_bounds__(kTopkThreads) select_topk(const __grid_constant__ PartialParams pp) {
+  __shared__ uint32_t keys[kTopkSmemKeys];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_digit, s_remaining;
-  __shared__ uint32_t scan_eq[kTopkThreads / 32], scan_sel[kTopkThreads / 32];
+  __shared__ uint32_t scan_eq[kTopkThreads / 32], scan_gt[kTopkThreads / 32];
   __shared__ int s_bad;
   const Shape &sh = pp.sh;
   const SelectArgs &a = pp.a;
@@ -262,91 +356,123 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk(const PartialParams 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, sh.P, a.status, false);
   const int np = (n + sh.P - 1) / sh.P;
-  int kp = a.topk[s] / sh.P;
-  if (tid == 0) s_bad = 0;
-  __syncthreads();
-  if (kp > sh.kmax || kp < 0 || a.topk[s] % sh.P != 0) {
+  const int topk_tokens = a.topk[s];
+  int kp = topk_tokens / sh.P;
+  if (kp > sh.kmax || kp < 0 || topk_tokens % sh.P != 0) {
     if (tid == 0) raise_status(a.status, kStatusBadIndex);
     kp = max(0, min(kp, sh.kmax));
   }
   const float *sc = a.scores + sh_idx * sh.max_pages;
   int32_t *out = a.idx_out + sh_idx * sh.kmax;
   const int take = min(kp, np);
-
-  // non-finite scores are reported (they come from non-finite inputs)
-  for (int i = tid; i < np; i += kTopkThreads)
-    if (!isfinite(sc[i])) s_bad = 1;
+  const bool staged = np <= kTopkSmemKeys;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  int bad = 0;
+  for (int i = tid; i < np; i += kTopkThreads) {
+    const float v = sc[i];
+    bad |= !isfinite(v);
+    if (staged) keys[i] = score_key(v);
+  }
+  if (bad) s_bad = 1;
   __syncthreads();
   if (s_bad && tid == 0) raise_status(a.status, kStatusNonfinite);
+  auto key_at = [&](int i) -> uint32_t { return staged ? keys[i] : score_key(sc[i]); };
 
   if (take >= np) {  // the budget covers the prefix: every page
     for (int i = tid; i < sh.kmax; i += kTopkThreads) out[i] = i < np ? i : -1;
     if (tid == 0) a.cnt_out[sh_idx] = np;
     return;
   }
-  // radix select of the take-th largest key, 8 bits at a time from the top
   uint32_t prefix = 0, mask = 0;
   if (tid == 0) s_remaining = (uint32_t)take;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
+    if (tid < 256) hist[tid] = 0;
     __syncthreads();
     for (int i = tid; i < np; i += kTopkThreads) {
-      const uint32_t key = score_key(sc[i]);
+      const uint32_t key = key_at(i);
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      uint32_t cum = 0, rem = s_remaining;
-      int dgt = 255;
-      for (; dgt > 0; --dgt) {
-        if (cum + hist[dgt] >= rem) break;
-        cum += hist[dgt];
+    if (warp == 0) {
+      // lane L owns bins 255-8L down to 248-8L; counts above a lane's bins are
+      // the exclusive prefix over the lanes before it
+      const uint32_t rem = s_remaining;
+      uint32_t cnt[8], local = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        cnt[q] = hist[255 - 8 * lane - q];
+        local += cnt[q];
       }
-      s_digit = (uint32_t)dgt;
-      s_remaining = rem - cum;
+      uint32_t incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const uint32_t above = incl - local;
+      if (above < rem && rem <= incl) {
+        uint32_t cum = above;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (cum + cnt[q] >= rem) {
+            s_digit = (uint32_t)(255 - 8 * lane - q);
+            s_remaining = rem - cum;
+            break;
+          }
+          cum += cnt[q];
+        }
+      }
     }
     __syncthreads();
     prefix |= s_digit << shift;
     mask |= 255u << shift;
-    __syncthreads();
   }
-  const uint32_t thr = prefix;           // value of the take-th largest key
+  const uint32_t thr = prefix;           // the take-th largest key
   const uint32_t need_eq = s_remaining;  // keys equal to thr to keep, lowest pages first
 
-  // ordered compaction: contiguous chunk per thread, block-wide exclusive scans
+  // ordered compaction: a contiguous chunk per thread, block-wide exclusive scans
   const int chunk = (np + kTopkThreads - 1) / kTopkThreads;
   const int i0 = min(np, tid * chunk), i1 = min(np, i0 + chunk);
   uint32_t n_eq = 0, n_gt = 0;
   for (int i = i0; i < i1; ++i) {
-    const uint32_t key = score_key(sc[i]);
+    const uint32_t key = key_at(i);
     n_gt += key > thr;
     n_eq += key == thr;
   }
-  // warp-inclusive scans of (n_eq, n_gt)
   uint32_t e = n_eq, g = n_gt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t e2 = __shfl_up_sync(0xffffffffu, e, o), g2 = __shfl_up_sync(0xffffffffu, g, o);
-    if (lane >= o) { e += e2; g += g2; }
+    if (lane >= o) {
+      e += e2;
+      g += g2;
+    }
   }
-  if (lane == 31) { scan_eq[warp] = e; scan_sel[warp] = g; }
+  if (lane == 31) {
+    scan_eq[warp] = e;
+    scan_gt[warp] = g;
+  }
   __syncthreads();
   if (warp == 0) {
-    uint32_t we = scan_eq[lane], wg = scan_sel[lane];
+    uint32_t we = scan_eq[lane], wg = scan_gt[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t e2 = __shfl_up_sync(0xffffffffu, we, o), g2 = __shfl_up_sync(0xffffffffu, wg, o);
-      if (lane >= o) { we += e2; wg += g2; }
+      if (lane >= o) {
+        we += e2;
+        wg += g2;
+      }
     }
     scan_eq[lane] = we;
-    scan_sel[lane] = wg;
+    scan_gt[lane] = wg;
   }
   __syncthreads();
   uint32_t eq_before = e - n_eq + (warp > 0 ? scan_eq[warp - 1] : 0u);
-  uint32_t gt_before = g - n_gt + (warp > 0 ? scan_sel[warp - 1] : 0u);
-  // position = selected pages before i = (greater before) + min(equal before, need_eq)
+  uint32_t gt_before = g - n_gt + (warp > 0 ? scan_gt[warp - 1] : 0u);
+  // position of a kept page = kept pages before it = (greater before) + min(equal before, need_eq)
   for (int i = i0; i < i1; ++i) {
-    const uint32_t key = score_key(sc[i]);
+    const uint32_t key = key_at(i);
     if (key > thr) {
       out[gt_before + min(eq_before, need_eq)] = i;
       ++gt_before;
@@ -369,13 +495,18 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
   if (err != cudaSuccess) return err;
   err = make_kv_tensor_map(&vmap, a.v, rows, D, PAGE);
   if (err != cudaSuccess) return err;
+  CUtensorMap kmap4, vmap4;
+  err = make_kv_pages_tensor_map(&kmap4, a.k, sh.n_phys, sh.Hkv, PAGE, D, tc::kBN / PAGE);
+  if (err != cudaSuccess) return err;
+  err = make_kv_pages_tensor_map(&vmap4, a.v, sh.n_phys, sh.Hkv, PAGE, D, tc::kBN / PAGE);
+  if (err != cudaSuccess) return err;
   constexpr auto kern = select_partial<D, PAGE>;
   constexpr size_t smem = tc::Layout<D, kSelStages>::kAlloc;
   err = set_smem_once<kern>(smem);
   if (err != cudaSuccess) return err;
   dim3 grid(plan.splits * plan.rowtiles, sh.Hkv, sh.S);
-  kern<<<grid, tc::kThreads, smem, stream>>>(pp, kmap, vmap);
-  const int score_ctas = (sh.max_pages + kPagesPerFinCta - 1) / kPagesPerFinCta;
+  kern<<<grid, tc::kThreads, smem, stream>>>(pp, kmap, vmap, kmap4, vmap4);
+  const int score_ctas = (sh.max_pages + plan.fin_pages - 1) / plan.fin_pages;
   const int o_ctas = (sh.BG + kRowsPerFinCta - 1) / kRowsPerFinCta;
   select_finalize<D, PAGE><<<dim3(score_ctas + o_ctas, sh.Hkv, sh.S), kFinThreads, 0, stream>>>(pp);
   select_topk<<<dim3(sh.Hkv, sh.S), kTopkThreads, 0, stream>>>(pp);
@@ -384,22 +515,31 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
 
 }  // namespace
 
+DSA_TRACE_EXPORT(dsa_trace_select)
+
 SelectPlan plan_select(const Shape &sh, int num_sms) {
   SelectPlan p{};
   p.rowtiles = (sh.BG + kRowsPerCta - 1) / kRowsPerCta;
   p.max_tiles = (int)(((long long)sh.max_pages * sh.P + tc::kBN - 1) / tc::kBN);
   const long long base = (long long)sh.S * sh.Hkv * p.rowtiles;
-  const long long target = num_sms;  // one resident CTA per SM
-  int splits = (int)std::max(1LL, (target + base - 1) / base);
+  // one resident CTA per SM and a single wave: a second, partial wave would
+  // double the makespan
+  int splits = (int)std::max(1LL, (long long)num_sms / base);
   splits = std::min(splits, p.max_tiles);
   p.tiles_per_split = (p.max_tiles + splits - 1) / splits;
   p.splits = (p.max_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
   auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
   size_t off = 4096;  // status word and counters
   const size_t shn = (size_t)sh.S * sh.Hkv;
+  // score CTAs of the finalize pass: about two per SM, each a multiple of 8 tiles
+  const long long all_pages = (long long)sh.S * sh.Hkv * sh.max_pages;
+  long long fp = (all_pages + 2LL * num_sms - 1) / (2LL * num_sms);
+  const long long tile_pages = tc::kBN / sh.P;  // score CTAs start on tile boundaries
+  p.fin_pages = (int)std::max(tile_pages * 8, (fp + tile_pages * 8 - 1) / (tile_pages * 8) * (tile_pages * 8));
   p.off_part_o = off;   off = align(off + shn * p.splits * sh.BG * sh.d * 4);
   p.off_part_ml = off;  off = align(off + shn * p.splits * sh.BG * 2 * 4);
-  p.off_pagepart = off; off = align(off + shn * sh.max_pages * sh.BG * 4);
+  const size_t units_per_page = sh.P > tc::kHalfBN ? (size_t)sh.P / tc::kHalfBN : 1;
+  p.off_pagepart = off; off = align(off + shn * sh.max_pages * units_per_page * sh.BG * 4);
   p.off_mtile = off;    off = align(off + shn * p.max_tiles * sh.BG * 4);
   p.off_scores = off;   off = align(off + shn * sh.max_pages * 4);
   p.total = off;

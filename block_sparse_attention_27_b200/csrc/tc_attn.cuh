@@ -1,18 +1,23 @@
 // tc_attn.cuh -- the tcgen05 attention engine shared by the selection and the
 // sparse pass: one CTA runs up to 128 query rows of one KV head against a list
-// of 64-token key tiles that a Policy describes.
+// of 64-key tiles that a Policy describes.
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: Policy::load_tile issues the tile's K and V boxes
 //               into a STAGES-deep ring of 128-byte-swizzled shared tiles;
 //   warp 1      TMEM owner and MMA issuer: S_k = Q K_k^T into a double-buffered
 //               TMEM S (64 fp32 columns each), O += P_k V_k into TMEM O;
-//   warps 2..5  one query row per thread (TMEM lane = row): online softmax in the
-//               log2 domain with lazy rescaling (the reference max moves only
-//               when a tile beats it by more than 2^8), per-page sums handed to
+//   warps 2..9  two softmax warpgroups that take alternate tiles (group g
+//               the tiles k with k % 2 == g), so that one group's exp phase
+//               overlaps the other's loads and stores.  Thread (g, r) owns query
+//               row r (TMEM lane r): online softmax in the log2 domain with lazy
+//               rescaling (the reference max moves only when a tile beats it by
+//               more than 2^8), per-unit sums (32 keys at most) handed to
 //               Policy::after_tile, P in bf16 to shared memory for the PV MMA.
-// After run() the softmax threads hold (m, l) of their row and O sits in TMEM;
-// the kernel reads it (Engine::load_o) and then calls Engine::teardown.
+//               Each group accumulates into its own TMEM O.
+// After run() every softmax thread holds its group's (m, l); finish() joins the
+// two groups' statistics, and the kernel combines the two O accumulators
+// (load_o) with the weights it returns before calling teardown().
 //
 // Every wait is time-bounded (sm100::mbar_wait); a timeout aborts the CTA,
 // which still drains its copies and MMAs before TMEM is freed.
@@ -20,13 +25,25 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "trace.cuh"
 
 namespace dsa {
 namespace tc {
 
 constexpr int kBN = 64;          // keys per tile
-constexpr int kThreads = 192;    // 6 warps
+constexpr int kHalfBN = kBN / 2; // keys per softmax warpgroup
+constexpr int kThreads = 320;    // 10 warps
+constexpr int kSoftmaxThreads = 256;
 constexpr float kRescaleLog2 = 8.f;
+
+// The unit of the per-page partial sums: min(PAGE, 32) keys of one page (a
+// 64-token page is two units).
+template <int PAGE>
+struct Units {
+  static constexpr int kKeys = PAGE < kHalfBN ? PAGE : kHalfBN;   // keys per unit
+  static constexpr int kPerTile = kBN / kKeys;                     // units per tile
+  static constexpr int kPerPage = PAGE / kKeys;                    // units per page
+};
 
 template <int D, int STAGES>
 struct Layout {
@@ -40,12 +57,15 @@ struct Layout {
   static constexpr uint32_t kOffKV = kOffQ + kHalves * kQHalf;
   static constexpr uint32_t kOffP = kOffKV + STAGES * kStageBytes;
   static constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
-  static constexpr int kNumBars = 2 * STAGES + 10;
+  static constexpr int kNumBars = 2 * STAGES + 15;  // the last one is the kernel's own
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kOffML = kOffQ;  // [2 groups][128] (m, l), once Q is dead
   static constexpr uint32_t kBytes = kOffMisc + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // room to align the base to 1 KB
-  static constexpr uint32_t kTmemCols = 256;         // S0 [0,64) S1 [64,128) O [128,128+D)
-  static constexpr uint32_t kTmemO = 128;
+  // TMEM: four S buffers of 64 columns (two per softmax group: buffer 2g+i),
+  // then the O accumulators of group 0 and group 1
+  static constexpr uint32_t kTmemO = 4 * kBN;
+  static constexpr uint32_t kTmemCols = 512;
   static_assert(D == 64 || D == 128, "head dimension");
 };
 
@@ -61,41 +81,77 @@ struct Engine {
   __device__ __forceinline__ uint32_t bar(int i) const { return base + L::kOffBar + 8u * (uint32_t)i; }
   __device__ __forceinline__ uint32_t kv_full(int st) const { return bar(st); }
   __device__ __forceinline__ uint32_t kv_empty(int st) const { return bar(STAGES + st); }
-  __device__ __forceinline__ uint32_t s_full(int b) const { return bar(2 * STAGES + b); }
-  __device__ __forceinline__ uint32_t s_free(int b) const { return bar(2 * STAGES + 2 + b); }
-  __device__ __forceinline__ uint32_t p_full(int b) const { return bar(2 * STAGES + 4 + b); }
-  __device__ __forceinline__ uint32_t pv_done(int b) const { return bar(2 * STAGES + 6 + b); }
-  __device__ __forceinline__ uint32_t q_full() const { return bar(2 * STAGES + 8); }
-  __device__ __forceinline__ uint32_t drain() const { return bar(2 * STAGES + 9); }
+  __device__ __forceinline__ uint32_t s_full(int sb) const { return bar(2 * STAGES + sb); }
+  __device__ __forceinline__ uint32_t s_free(int sb) const { return bar(2 * STAGES + 4 + sb); }
+  __device__ __forceinline__ uint32_t p_full(int g) const { return bar(2 * STAGES + 8 + g); }
+  __device__ __forceinline__ uint32_t pv_done(int g) const { return bar(2 * STAGES + 10 + g); }
+  __device__ __forceinline__ uint32_t q_full() const { return bar(2 * STAGES + 12); }
+  __device__ __forceinline__ uint32_t drain() const { return bar(2 * STAGES + 13); }
+  __device__ __forceinline__ uint32_t user_bar() const { return bar(2 * STAGES + 14); }
+  // tile k runs on softmax group k % 2 as that group's (k / 2)-th tile, in S buffer
+  // 2 * group + (k / 2) % 2
+  static __device__ __forceinline__ int s_buf(int k) { return 2 * (k & 1) + ((k >> 1) & 1); }
   __device__ __forceinline__ uint32_t stage_k(int st) const { return base + L::kOffKV + st * L::kStageBytes; }
   __device__ __forceinline__ uint32_t stage_v(int st) const { return stage_k(st) + L::kKBytes; }
   __device__ __forceinline__ volatile int *abort_flag() const {
     return reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
   }
 
-  // Barrier init and TMEM allocation; every thread of the CTA calls it.
-  __device__ __forceinline__ void init(unsigned char *smem_raw, uint32_t *status) {
+  // Softmax-thread geometry --------------------------------------------------
+  __device__ __forceinline__ int quarter() const { return warp & 3; }
+  __device__ __forceinline__ int row_in_tile() const { return quarter() * 32 + lane; }
+  __device__ __forceinline__ int group() const { return (warp - 2) >> 2; }  // softmax group 0 or 1
+  __device__ __forceinline__ uint32_t lane_tmem() const { return tmem + ((uint32_t)(quarter() * 32) << 16); }
+
+  // Barrier init and TMEM allocation; every thread of the CTA calls it.  The
+  // softmax threads already copy their query rows into the Q tile, and (for a
+  // policy that allows it) the producer issues the loads of the first STAGES
+  // tiles, before the CTA-wide barrier.
+  template <class Policy>
+  __device__ __forceinline__ void init(unsigned char *smem_raw, uint32_t *status, Policy &pol,
+                                       int num_tiles) {
     using namespace sm100;
     const uint32_t raw = smem_addr(smem_raw);
     base = (raw + 1023u) & ~1023u;
     smem = smem_raw + (base - raw);
     warp = threadIdx.x >> 5;
     lane = threadIdx.x & 31;
+    pol.prepare(smem);  // per-CTA tables of the policy (all threads)
+    if (warp >= 2) {    // half of this row's query into the swizzled Q tile (zeros past the end)
+      const int r = row_in_tile();
+      constexpr int kChunks = D / 16;  // 16-byte chunks per half row
+      const int c0 = group() * kChunks;
+      const uint4 *src = reinterpret_cast<const uint4 *>(pol.q_row(r));
+      uint4 v[kChunks];
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) v[i] = src ? __ldg(src + c0 + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int c = c0 + i;
+        *reinterpret_cast<uint4 *>(smem + L::kOffQ + (c >> 3) * L::kQHalf + sw128_offset(r, c & 7)) = v[i];
+      }
+      fence_proxy_async_smem();
+    }
     if (threadIdx.x == 0) {
       for (int st = 0; st < STAGES; ++st) {
         mbar_init(kv_full(st), 1);
         mbar_init(kv_empty(st), 1);
       }
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(s_full(b), 1);
-        mbar_init(s_free(b), 128);
-        mbar_init(p_full(b), 128);
-        mbar_init(pv_done(b), 1);
+      for (int sb = 0; sb < 4; ++sb) {
+        mbar_init(s_full(sb), 1);
+        mbar_init(s_free(sb), kSoftmaxThreads / 2);
       }
-      mbar_init(q_full(), 128);
+      for (int g = 0; g < 2; ++g) {
+        mbar_init(p_full(g), kSoftmaxThreads / 2);
+        mbar_init(pv_done(g), 1);
+      }
+      mbar_init(q_full(), kSoftmaxThreads);
       mbar_init(drain(), 1);
+      mbar_init(user_bar(), 1);
       *abort_flag() = 0;
       fence_mbar_init();
+      // thread 0 is the producer: the first tiles' loads go out right away
+      if (Policy::kIssueBeforeSync && num_tiles > 0) issue_first(pol, num_tiles);
     }
     if (warp == 1) {
       tmem_alloc(base + L::kOffMisc, L::kTmemCols);
@@ -104,19 +160,30 @@ struct Engine {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // (a policy whose tile addresses come from a table built in prepare()
+    // issues its first loads once that table is complete)
+    if (!Policy::kIssueBeforeSync && threadIdx.x == 0 && num_tiles > 0) issue_first(pol, num_tiles);
     tmem = *reinterpret_cast<volatile uint32_t *>(smem + L::kOffMisc);
     ctx = sm100::WaitCtx{abort_flag(), status};
+    if (warp >= 2) mbar_arrive(q_full());
+    if (threadIdx.x == 0) DSA_TRACE_EVENT(1);
   }
 
-  // Softmax-thread helpers --------------------------------------------------
-  __device__ __forceinline__ int row_in_tile() const { return (warp & 3) * 32 + lane; }
-  __device__ __forceinline__ uint32_t lane_tmem() const { return tmem + ((uint32_t)((warp & 3) * 32) << 16); }
+  template <class Policy>
+  __device__ __forceinline__ void issue_first(Policy &pol, int num_tiles) {
+    pol.prefetch();
+    for (int k = 0; k < min(STAGES, num_tiles); ++k)
+      pol.load_tile(k, stage_k(k), stage_v(k), L::kKVHalf, kv_full(k));
+    DSA_TRACE_EVENT(2);
+  }
 
   // Runs the pipeline over `num_tiles` tiles.  Softmax threads return their
-  // row's (m, l) in the log2 domain and whether the CTA is still alive.
+  // row's (m, l) in the log2 domain (l over both halves) and whether the CTA is
+  // still alive.
   template <int PAGE, class Policy>
   __device__ __forceinline__ bool run(Policy &pol, int num_tiles, float &m_out, float &l_out) {
     using namespace sm100;
+    using U = Units<PAGE>;
     volatile int never = 0;
     const WaitCtx drain_ctx{&never, ctx.status};
     bool alive = true;
@@ -125,12 +192,12 @@ struct Engine {
     if (warp == 0) {
       // ---------------------------------------------------------- producer --
       if (lane == 0 && num_tiles > 0) {
-        pol.prefetch();
-        int issued = 0;
-        for (int k = 0; k < num_tiles; ++k) {
+        int issued = min(STAGES, num_tiles);  // issued during init
+        for (int k = issued; k < num_tiles; ++k) {
           const int st = k % STAGES;
-          if (k >= STAGES && !mbar_wait(kv_empty(st), ((k / STAGES) - 1) & 1, ctx)) break;
+          if (!mbar_wait(kv_empty(st), ((k / STAGES) - 1) & 1, ctx)) break;
           pol.load_tile(k, stage_k(st), stage_v(st), L::kKVHalf, kv_full(st));
+          if (k == STAGES) DSA_TRACE_EVENT(24);
           issued = k + 1;
         }
         // copies in flight land before the CTA's shared memory is released
@@ -142,73 +209,99 @@ struct Engine {
       if (lane == 0 && num_tiles > 0) {
         constexpr uint32_t kIdS = idesc_bf16(128, kBN, false, false);
         constexpr uint32_t kIdO = idesc_bf16(128, D, false, true);
+        // S of tile j + kLook is issued before P of tile j is awaited, so that a
+        // softmax group finds its next S ready; kLook stays below STAGES because
+        // that tile's K/V stage is freed by PV_{j + kLook - STAGES}
+        constexpr int kLook = STAGES >= 3 ? 2 : 1;
+        auto issue_s = [&](int k) -> bool {
+          const int st = k % STAGES, sb = s_buf(k);
+          if (!mbar_wait(kv_full(st), (k / STAGES) & 1, ctx)) return false;
+          if (k == 0) DSA_TRACE_EVENT(3);
+          if (k >= 4 && !mbar_wait(s_free(sb), (((k >> 1) - 2) >> 1) & 1, ctx)) return false;
+          tc_fence_after();
+          const uint32_t sk = stage_k(st);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t hf = kk >> 2, sub = kk & 3;
+            const uint64_t ad = sdesc_sw128(base + L::kOffQ + hf * L::kQHalf + sub * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sk + hf * L::kKVHalf + sub * 32, 16, 1024);
+            umma_bf16(tmem + sb * kBN, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full(sb));
+          if (k == 1) DSA_TRACE_EVENT(25);
+          if (k == 4) DSA_TRACE_EVENT(15);
+          return true;
+        };
         bool ok = mbar_wait(q_full(), 0, ctx);
-        for (int k = 0; ok && k <= num_tiles; ++k) {
-          if (k < num_tiles) {
-            const int st = k % STAGES, b = k & 1;
-            if (!mbar_wait(kv_full(st), (k / STAGES) & 1, ctx)) break;
-            if (k >= 2 && !mbar_wait(s_free(b), ((k - 2) >> 1) & 1, ctx)) break;
-            tc_fence_after();
-            const uint32_t sk = stage_k(st);
+        DSA_TRACE_EVENT(12);
+        for (int k = 0; ok && k < kLook && k < num_tiles; ++k) ok = issue_s(k);
+        for (int j = 0; ok && j < num_tiles; ++j) {
+          if (j + kLook < num_tiles && !issue_s(j + kLook)) break;
+          const int st = j % STAGES, g = j & 1;
+          if (!mbar_wait(p_full(g), (j >> 1) & 1, ctx)) break;
+          if (j == 2) DSA_TRACE_EVENT(14);
+          tc_fence_after();
+          const uint32_t sv = stage_v(st);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t hf = kk >> 2, sub = kk & 3;
-              const uint64_t ad = sdesc_sw128(base + L::kOffQ + hf * L::kQHalf + sub * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sk + hf * L::kKVHalf + sub * 32, 16, 1024);
-              umma_bf16(tmem + b * kBN, ad, bd, kIdS, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(s_full(b));
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(base + L::kOffP + g * L::kPBytes + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sv + kk * 16 * 128, L::kKVHalf, 1024);
+            umma_bf16(tmem + L::kTmemO + g * D, ad, bd, kIdO, (j > 1 || kk > 0) ? 1u : 0u);
           }
-          if (k >= 1) {
-            const int j = k - 1, st = j % STAGES, b = j & 1;
-            if (!mbar_wait(p_full(b), (j >> 1) & 1, ctx)) break;
-            tc_fence_after();
-            const uint32_t sv = stage_v(st);
-#pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-              const uint64_t ad = sdesc_sw128(base + L::kOffP + b * L::kPBytes + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sv + kk * 16 * 128, L::kKVHalf, 1024);
-              umma_bf16(tmem + L::kTmemO, ad, bd, kIdO, (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(pv_done(b));
-            umma_commit(kv_empty(st));
-          }
+          umma_commit(pv_done(g));
+          umma_commit(kv_empty(st));
+          if (j == 0) DSA_TRACE_EVENT(26);
         }
         // every issued MMA completes before TMEM can be released
         umma_commit(drain());
         mbar_wait(drain(), 0, drain_ctx);
       }
     } else {
-      // ------------------------------------------------------ softmax rows --
+      // ---------------------------------------------------- softmax groups --
       const int r = row_in_tile();
+      const int g = group();
       const uint32_t lt = lane_tmem();
-      {  // this row's query into the swizzled Q tile (zeros for rows past the end)
-        const uint4 *src = reinterpret_cast<const uint4 *>(pol.q_row(r));
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 v = src ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4 *>(smem + L::kOffQ + (c >> 3) * L::kQHalf + sw128_offset(r, c & 7)) = v;
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(q_full());
-      }
+      const uint32_t o_col = L::kTmemO + g * D;
       float m_used = -INFINITY, l = 0.f;
-      for (int k = 0; k < num_tiles; ++k) {
-        const int st = k % STAGES, b = k & 1;
-        alive = __all_sync(0xffffffffu, mbar_wait(s_full(b), (k >> 1) & 1, ctx));
+      int mine = 0;  // tiles this group has finished
+      for (int k = g; k < num_tiles; k += 2, ++mine) {
+        const int st = k % STAGES, sb = s_buf(k);
+        alive = __all_sync(0xffffffffu, mbar_wait(s_full(sb), (mine >> 1) & 1, ctx));
         if (!alive) break;
+        const bool lead = r == 0;
+        const bool tr = k == 1 && lead;
+        if (k == 0 && lead) DSA_TRACE_EVENT(4);
+        if (tr) DSA_TRACE_EVENT(16);
+        if (k == 2 && lead) DSA_TRACE_EVENT(27);
+        if (k == 4 && lead) DSA_TRACE_EVENT(28);
         tc_fence_after();
         uint32_t sraw[kBN];
-        tmem_ld32(lt + b * kBN, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
-        tmem_ld32(lt + b * kBN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
-        uint64_t key_ok = pol.key_mask(k);  // bit j: key j of the tile takes part
-        float x[kBN];
-        float tmax = -INFINITY;
+        tmem_ld32(lt + sb * kBN, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
+        tmem_ld32(lt + sb * kBN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
+        if (tr) DSA_TRACE_EVENT(17);
+        const uint64_t key_ok = pol.key_mask(k);  // bit j: key j of the tile takes part
+        if (tr) DSA_TRACE_EVENT(18);
+        float x[kBN];  // raw logits q.k; keys that take no part become -inf
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (key_ok == ~0ull) {
 #pragma unroll
-        for (int j = 0; j < kBN; ++j) {
-          x[j] = ((key_ok >> j) & 1ull) ? __uint_as_float(sraw[j]) * pol.sl2 : -INFINITY;
-          tmax = fmaxf(tmax, x[j]);
+          for (int j = 0; j < kBN; ++j) {
+            x[j] = __uint_as_float(sraw[j]);
+            mx[j & 3] = fmaxf(mx[j & 3], x[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < kBN; ++j) {
+            x[j] = ((key_ok >> j) & 1ull) ? __uint_as_float(sraw[j]) : -INFINITY;
+            mx[j & 3] = fmaxf(mx[j & 3], x[j]);
+          }
         }
+        // tile max in the log2 domain (the scale is positive, so it commutes with max)
+        const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * pol.sl2;
+        if (tr) DSA_TRACE_EVENT(19);
+        // PV of this group's previous tile must have landed before O is rescaled
+        // or the group's P buffer is rewritten
+        bool pv_ready = mine == 0;
         const bool need = tmax > m_used + kRescaleLog2 || (m_used == -INFINITY && tmax > -INFINITY);
         if (__any_sync(0xffffffffu, need)) {
           float alpha = 1.f;
@@ -217,37 +310,39 @@ struct Engine {
             m_used = tmax;
             l *= alpha;
           }
-          if (k > 0) {  // O holds earlier tiles: let PV_{k-1} land, then scale it
-            alive = __all_sync(0xffffffffu, mbar_wait(pv_done((k - 1) & 1), ((k - 1) >> 1) & 1, ctx));
+          if (mine > 0) {  // O holds this group's earlier tiles: scale it
+            alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 1) & 1, ctx));
             if (!alive) break;
+            pv_ready = true;
             tc_fence_after();
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
               uint32_t o[32];
-              tmem_ld32(lt + L::kTmemO + c0, o);
+              tmem_ld32(lt + o_col + c0, o);
 #pragma unroll
               for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(lt + L::kTmemO + c0, o);
+              tmem_st32(lt + o_col + c0, o);
             }
           }
         }
         const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-        float psum[kBN / PAGE];
+        float usum[U::kPerTile];
 #pragma unroll
-        for (int pi = 0; pi < kBN / PAGE; ++pi) psum[pi] = 0.f;
+        for (int u = 0; u < U::kPerTile; ++u) usum[u] = 0.f;
 #pragma unroll
         for (int j = 0; j < kBN; ++j) {
-          const float p = fast_exp2(x[j] - mu);
+          const float p = fast_exp2(fmaf(x[j], pol.sl2, -mu));
           x[j] = p;
-          psum[j / PAGE] += p;
+          usum[j / U::kKeys] += p;
         }
 #pragma unroll
-        for (int pi = 0; pi < kBN / PAGE; ++pi) l += psum[pi];
-        if (k >= 2) {  // P buffer b was read by PV_{k-2}
-          alive = __all_sync(0xffffffffu, mbar_wait(pv_done(b), ((k - 2) >> 1) & 1, ctx));
+        for (int u = 0; u < U::kPerTile; ++u) l += usum[u];
+        if (tr) DSA_TRACE_EVENT(20);
+        if (!pv_ready) {
+          alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 1) & 1, ctx));
           if (!alive) break;
         }
-        unsigned char *prow = smem + L::kOffP + b * L::kPBytes;
+        unsigned char *prow = smem + L::kOffP + g * L::kPBytes;
 #pragma unroll
         for (int c = 0; c < kBN / 8; ++c) {
           uint4 v;
@@ -257,6 +352,7 @@ struct Engine {
           v.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
           *reinterpret_cast<uint4 *>(prow + sw128_offset(r, c)) = v;
         }
+        if (tr) DSA_TRACE_EVENT(21);
         // value rows of keys that take no part are zeroed so that 0 * stale data
         // cannot reach O (thread r < 64 looks after key r of the tile)
         if (r < kBN && !((key_ok >> r) & 1ull) && mbar_wait(kv_full(st), (k / STAGES) & 1, ctx)) {
@@ -267,27 +363,60 @@ struct Engine {
             for (int c = 0; c < 8; ++c)
               *reinterpret_cast<uint4 *>(vrow + hf * L::kKVHalf + c * 16) = make_uint4(0, 0, 0, 0);
         }
-        pol.after_tile(k, r, m_used, psum);
+        pol.after_tile(k, r, m_used, usum);
+        if (tr) DSA_TRACE_EVENT(22);
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(s_free(b));
-        mbar_arrive(p_full(b));
+        mbar_arrive(s_free(sb));
+        mbar_arrive(p_full(g));
+        if (tr) DSA_TRACE_EVENT(23);
+        if (k == 2 && lead) DSA_TRACE_EVENT(13);
+        if (k == 4 && lead) DSA_TRACE_EVENT(29);
+        if (k >= num_tiles - 2 && lead && g == ((num_tiles - 1) & 1)) DSA_TRACE_EVENT(5);
       }
-      if (alive && num_tiles > 0) {
-        const int j = num_tiles - 1;
-        alive = __all_sync(0xffffffffu, mbar_wait(pv_done(j & 1), (j >> 1) & 1, ctx));
+      if (alive && mine > 0) {  // the group's last PV has landed in its O
+        alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 1) & 1, ctx));
         if (alive) tc_fence_after();
+        if (r == 0 && g == ((num_tiles - 1) & 1)) DSA_TRACE_EVENT(6);
       }
       m_out = m_used;
-      l_out = l;
-      alive = alive && num_tiles > 0;
+      l_out = (alive && mine > 0) ? l : 0.f;
     }
     return alive;
   }
 
-  // 32 columns [c0, c0+32) of this softmax thread's O row (warp-collective).
-  __device__ __forceinline__ void load_o(int c0, uint32_t (&o)[32]) const {
-    sm100::tmem_ld32(lane_tmem() + L::kTmemO + c0, o);
+  // Joins the two softmax groups' statistics of each row; every thread of the
+  // CTA calls it (it contains a CTA barrier).  For softmax threads it returns
+  // the row's merged (m, l) and the weights wa, wb with which the groups' O
+  // accumulators combine: O = wa * O_0 + wb * O_1 (a weight is 0 for a group
+  // that saw no keys, whose accumulator holds no data).
+  __device__ __forceinline__ void finish(float m, float l, float &m_row, float &l_row, float &wa,
+                                         float &wb) {
+    float2 *ml = reinterpret_cast<float2 *>(smem + L::kOffML);
+    const int r = row_in_tile();
+    // both groups have seen their last PV complete, hence every MMA (which all
+    // read Q) is done: only then may the statistics area in the Q tile be written
+    __syncthreads();
+    if (warp >= 2) ml[group() * 128 + r] = make_float2(m, l);
+    __syncthreads();
+    m_row = -INFINITY;
+    l_row = 0.f;
+    wa = wb = 0.f;
+    if (warp >= 2) {
+      const float2 a = ml[r], b = ml[128 + r];
+      const float M = fmaxf(a.y > 0.f ? a.x : -INFINITY, b.y > 0.f ? b.x : -INFINITY);
+      wa = a.y > 0.f ? exp2f(a.x - M) : 0.f;
+      wb = b.y > 0.f ? exp2f(b.x - M) : 0.f;
+      m_row = M;
+      l_row = wa * a.y + wb * b.y;
+    }
+    __syncthreads();  // the statistics area (in the Q tile) may be reused after this
+  }
+
+  // 32 columns [c0, c0+32) of group `which`'s O accumulator for this thread's
+  // row (warp-collective).
+  __device__ __forceinline__ void load_o(int which, int c0, uint32_t (&o)[32]) const {
+    sm100::tmem_ld32(lane_tmem() + L::kTmemO + which * D + c0, o);
   }
 
   // All threads: waits for everybody, then the TMEM owner frees TMEM.

@@ -45,6 +45,23 @@ cudaError_t make_kv_tensor_map(CUtensorMap *out, const void *base, long long row
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// The same cache seen as 4-D (D, P, Hkv, n_phys): one box is 64 elements x P
+// tokens x 1 head x `pages` consecutive physical pages, i.e. `pages` whole pages
+// of one KV head in one load, landing as pages*P rows of 128 bytes.
+cudaError_t make_kv_pages_tensor_map(CUtensorMap *out, const void *base, long long n_phys, int Hkv,
+                                     int P, int D, int pages) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P, (cuuint64_t)Hkv, (cuuint64_t)n_phys};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)P * D * 2, (cuuint64_t)Hkv * P * D * 2};
+  cuuint32_t box[4] = {64u, (cuuint32_t)P, 1u, (cuuint32_t)pages};
+  cuuint32_t elem_strides[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                  box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // The block's own keys or values [S*B, Hkv, D] bf16 as a 3-D tensor (D, Hkv,
 // S*B); one box is 64 elements x 1 head x 64 tokens, so one load brings up to 64
 // consecutive tokens of one KV head (rows past S*B read as zeros).
