@@ -63,6 +63,7 @@ struct SelectPolicy {
     return (p >= 0 && p < n_phys) ? p : -1;
   }
   __device__ __forceinline__ void prepare(unsigned char *) const {}
+  __device__ __forceinline__ void ready() const {}
   __device__ __forceinline__ void prefetch() const {
     sm100::tma_prefetch_map(kmap);
     sm100::tma_prefetch_map(vmap);

@@ -5,13 +5,14 @@
 // tokens, with no mask inside the block.
 //
 // One launch per step.  A thread-block cluster of C CTAs serves one (sequence,
-// KV head, 128-row tile): CTA c runs the tcgen05 engine (tc_attn.cuh) over its
-// slice [c*ppc, (c+1)*ppc) of the selected pages, gathered page by page with TMA
-// through the page table; the last CTA also takes the block's own tokens
-// (a 3-D TMA box over blk_k / blk_v).  The C partial results (unnormalised O in
-// shared memory, row max m and sum l) are merged through distributed shared
-// memory: after a cluster barrier CTA c reads every CTA's (m, l, O) for its
-// share of the rows and writes those rows of o_out in bf16.
+// KV head, 128-row tile): CTAs 0..C-2 run the tcgen05 engine (tc_attn.cuh) over
+// their slices [c*ppc, (c+1)*ppc) of the selected pages, gathered with TMA
+// through the page table; CTA C-1 takes the block's own tokens (a 3-D TMA box
+// over blk_k / blk_v), so that no CTA carries both.  The C partial results are
+// then merged inside the cluster: every CTA pushes each owner CTA the rows that
+// owner writes (its normalised output rows in fp16 plus the row max and sum),
+// with bulk copies into the owner's receive buffer, and each owner combines the
+// C contributions of its rows and writes them to o_out in bf16.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -27,26 +28,30 @@ constexpr int kSpStages = 2;
 constexpr int kRowsPerCta = 128;
 constexpr int kMaxCluster = 16;
 
-// Exchange buffers of the cluster merge.  A row is the CTA's normalised output
-// row O/l in fp16 (D values) followed by (m, l, -, -) in fp32; the receive
-// buffer (128 rows: rpc rows from each of the C CTAs) lies after every region
-// the attention engine uses, so data from a CTA that finished early cannot
-// land on tiles that are still being read.
+// Exchange buffers of the cluster merge.  A row is a CTA's normalised output row
+// O/l in fp16 (D values) followed by (m, l, -, -) in fp32.  CTA j owns rows
+// [j*rpc, min(128, (j+1)*rpc)) with rpc = ceil(128 / C); its receive buffer has
+// one slot of rpc rows per source CTA and lies after every region the attention
+// engine uses, so data from a CTA that finished early cannot land on tiles that
+// are still being read.  The merge weights (one per owned row and source) and
+// the CTA's page table follow it.
 template <int D>
 struct MergeLayout {
   static constexpr uint32_t kRowBytes = D * 2 + 16;
-  template <int STAGES>
-  static constexpr uint32_t kRecvOffset() {
-    return (tc::Layout<D, STAGES>::kBytes + 1023u) & ~1023u;
+  static __host__ __device__ constexpr uint32_t recv_offset() {
+    return (tc::Layout<D, kSpStages>::kBytes + 1023u) & ~1023u;
   }
-  // the page table of the CTA's selected entries (int2 each) follows
-  template <int STAGES>
-  static constexpr uint32_t kTableOffset() {
-    return kRecvOffset<STAGES>() + 128u * kRowBytes;
+  static __host__ __device__ constexpr uint32_t rpc(int C) { return (kRowsPerCta + C - 1) / C; }
+  static __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
+  static __host__ __device__ constexpr uint32_t weights_offset(int C) {
+    return align16(recv_offset() + (uint32_t)C * rpc(C) * kRowBytes);
   }
-  template <int STAGES>
-  static constexpr size_t kSmem(int ppc) {
-    return kTableOffset<STAGES>() + 8u * (uint32_t)ppc + 1024u;  // + alignment slack
+  // int2 entries: the offset must stay 8-byte (here 16-byte) aligned whatever C is
+  static __host__ __device__ constexpr uint32_t table_offset(int C) {
+    return align16(weights_offset(C) + (uint32_t)(rpc(C) * C + 16) * 4u);
+  }
+  static __host__ __device__ constexpr size_t smem(int C, int ppc) {
+    return table_offset(C) + 8u * (uint32_t)ppc + 1024u;  // + alignment slack
   }
 };
 
@@ -58,9 +63,10 @@ struct SparseParams {
 
 template <int D, int PAGE>
 struct SparsePolicy {
-  // the CTA's selected pages are resolved once (prepare) into a shared-memory
-  // table of (logical page, physical page); the first loads wait for it
-  static constexpr bool kIssueBeforeSync = false;
+  // the CTA's selected pages are resolved into a shared-memory table of
+  // (logical page, physical page) during set-up; until that table is complete
+  // (only the producer's first loads) entries are read directly
+  static constexpr bool kIssueBeforeSync = true;
   static constexpr int kPagesPerTile = tc::kBN / PAGE;
   const CUtensorMap *kmap, *vmap, *kmap4, *vmap4, *bkmap, *bvmap;
   const int32_t *idx_row;       // idx[s, h, :]
@@ -69,24 +75,31 @@ struct SparsePolicy {
   uint32_t *status;
   const int2 *tab;              // shared: (lp, phys) per entry of this CTA, phys < 0 = unusable
   uint32_t tab_off;             // byte offset of the table in the aligned shared memory
+  bool table_ready;
   long long n_phys, phys0;
   int Hkv, h, G, Hq, B, BG, s, n, np, e_begin, e_end, sel_tiles, row_base;
   float sl2;
 
+  __device__ __forceinline__ int2 resolve(int e) const {
+    const int lp = idx_row[e];
+    int phys = -1;
+    if (lp >= 0 && lp < np) {
+      const long long p = page_row ? (long long)page_row[lp] : phys0 + lp;
+      if (p >= 0 && p < n_phys) phys = (int)p;
+    }
+    return make_int2(lp, phys);
+  }
   __device__ __forceinline__ void prepare(unsigned char *smem) {
     int2 *t = reinterpret_cast<int2 *>(smem + tab_off);
     for (int e = e_begin + (int)threadIdx.x; e < e_end; e += (int)blockDim.x) {
-      const int lp = idx_row[e];
-      int phys = -1;
-      if (lp >= 0 && lp < np) {
-        const long long p = page_row ? (long long)page_row[lp] : phys0 + lp;
-        if (p >= 0 && p < n_phys) phys = (int)p;
-      }
-      if (phys < 0) raise_status(status, kStatusBadIndex);
-      t[e - e_begin] = make_int2(lp, phys);
+      const int2 v = resolve(e);
+      if (v.y < 0) raise_status(status, kStatusBadIndex);
+      t[e - e_begin] = v;
     }
     tab = t;
+    table_ready = false;
   }
+  __device__ __forceinline__ void ready() { table_ready = true; }
   __device__ __forceinline__ void prefetch() const {
     sm100::tma_prefetch_map(kmap);
     sm100::tma_prefetch_map(vmap);
@@ -96,7 +109,8 @@ struct SparsePolicy {
     sm100::tma_prefetch_map(bvmap);
   }
   __device__ __forceinline__ int2 entry(int e) const {
-    return e < e_end ? tab[e - e_begin] : make_int2(-1, -1);
+    if (e >= e_end) return make_int2(-1, -1);
+    return table_ready ? tab[e - e_begin] : resolve(e);
   }
   __device__ __forceinline__ void load_tile(int k, uint32_t sk, uint32_t sv, uint32_t half_bytes,
                                             uint32_t bar) const {
@@ -172,7 +186,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kmap4,
                 const __grid_constant__ CUtensorMap vmap4, const __grid_constant__ CUtensorMap bkmap,
                 const __grid_constant__ CUtensorMap bvmap) {
-  using L = tc::Layout<D, kSpStages>;
+  using M = MergeLayout<D>;
   extern __shared__ unsigned char smem_raw[];
   const Shape &sh = prm.sh;
   const SparsePlan &plan = prm.plan;
@@ -189,10 +203,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     if (reporter) raise_status(a.status, kStatusBadIndex);
     cnt = max(0, min(cnt, sh.kmax));
   }
-  const int e_begin = min(cnt, c * plan.ppc), e_end = min(cnt, (c + 1) * plan.ppc);
+  // CTAs 0..C-2: pages; CTA C-1: the block's own tokens
+  const bool blk_cta = c == C - 1;
+  const int e_begin = blk_cta ? cnt : min(cnt, c * plan.ppc);
+  const int e_end = blk_cta ? cnt : min(cnt, (c + 1) * plan.ppc);
   constexpr int kPagesPerTile = tc::kBN / PAGE;
   const int sel_tiles = (e_end - e_begin + kPagesPerTile - 1) / kPagesPerTile;
-  const int num_tiles = sel_tiles + (c == C - 1 ? plan.blk_tiles : 0);
+  const int num_tiles = sel_tiles + (blk_cta ? plan.blk_tiles : 0);
   const int row_base = rt * kRowsPerCta;
 
   SparsePolicy<D, PAGE> pol;
@@ -207,7 +224,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
   pol.status = a.status;
   pol.tab = nullptr;
-  pol.tab_off = MergeLayout<D>::template kTableOffset<kSpStages>();
+  pol.tab_off = M::table_offset(C);
+  pol.table_ready = false;
   pol.n_phys = sh.n_phys;
   pol.phys0 = (long long)s * sh.max_pages;
   pol.Hkv = sh.Hkv;
@@ -227,10 +245,12 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
   tc::Engine<D, kSpStages> eng;
   eng.init(smem_raw, a.status, pol, num_tiles);
-  // this CTA will receive one slice of rpc rows from every CTA of the cluster
-  using M = MergeLayout<D>;
-  const int rpc = kRowsPerCta / C;  // C is a power of two <= 16
-  if (threadIdx.x == 0) sm100::mbar_arrive_expect_tx(eng.user_bar(), kRowsPerCta * M::kRowBytes);
+  // rows this CTA owns in the merge, and the bytes it will receive for them
+  const int rpc = (int)M::rpc(C);
+  const int r0 = c * rpc;
+  const int nrows = max(0, min(kRowsPerCta, r0 + rpc) - r0);
+  if (threadIdx.x == 0)
+    sm100::mbar_arrive_expect_tx(eng.user_bar(), (uint32_t)(C * nrows) * M::kRowBytes);
   sm100::cluster_arrive();  // barrier init and expected bytes are visible to the cluster
 
   float m, l;
@@ -278,13 +298,17 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   __syncthreads();
   sm100::cluster_wait();  // every CTA of the cluster has armed its receive barrier
   if (threadIdx.x == 0) DSA_TRACE_EVENT(8);
-  const uint32_t recv = eng.base + M::template kRecvOffset<kSpStages>();
+  const uint32_t recv = eng.base + M::recv_offset();
   if (threadIdx.x == 0) {
     const uint32_t send = smem_addr(sendb);
-    for (int j = 0; j < C; ++j)
+    for (int j = 0; j < C; ++j) {
+      const int jr0 = j * rpc;
+      const int jn = max(0, min(kRowsPerCta, jr0 + rpc) - jr0);
+      if (jn == 0) continue;
       sm100::bulk_copy_to_cluster(sm100::cluster_map(recv + c * rpc * M::kRowBytes, j),
-                                  send + j * rpc * M::kRowBytes, rpc * M::kRowBytes,
+                                  send + jr0 * M::kRowBytes, jn * M::kRowBytes,
                                   sm100::cluster_map(eng.user_bar(), j));
+    }
     sm100::bulk_commit();
   }
 
@@ -292,26 +316,34 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const bool got = __syncthreads_and(sm100::mbar_wait(eng.user_bar(), 0, eng.ctx));
   if (threadIdx.x == 0) DSA_TRACE_EVENT(9);
   const int rows_here = min(kRowsPerCta, sh.BG - row_base);
-  const int r0 = c * rpc;
-  const unsigned char *rb = eng.smem + M::template kRecvOffset<kSpStages>();
-  constexpr int kChunks = D / 8;  // 8 values (16 bytes of fp16) per work item
-  for (int t = threadIdx.x; got && t < rpc * kChunks; t += blockDim.x) {
-    const int rl = t / kChunks, ch = t % kChunks;
-    if (r0 + rl >= rows_here) continue;
+  const unsigned char *rb = eng.smem + M::recv_offset();
+  float *wts = reinterpret_cast<float *>(eng.smem + M::weights_offset(C));  // [nrows][C]
+  for (int rl = threadIdx.x; got && rl < nrows; rl += blockDim.x) {
     float mx = -INFINITY;
     for (int j = 0; j < C; ++j) {
       const float2 st = *reinterpret_cast<const float2 *>(rb + (j * rpc + rl) * M::kRowBytes + D * 2);
       if (st.y > 0.f) mx = fmaxf(mx, st.x);
     }
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     float lsum = 0.f;
     for (int j = 0; j < C; ++j) {
-      const unsigned char *src = rb + (j * rpc + rl) * M::kRowBytes;
-      const float2 st = *reinterpret_cast<const float2 *>(src + D * 2);
-      if (!(st.y > 0.f)) continue;  // an empty partial
-      const float w = exp2f(st.x - mx) * st.y;
+      const float2 st = *reinterpret_cast<const float2 *>(rb + (j * rpc + rl) * M::kRowBytes + D * 2);
+      const float w = st.y > 0.f ? exp2f(st.x - mx) * st.y : 0.f;  // 0: an empty partial
+      wts[rl * C + j] = w;
       lsum += w;
-      const uint4 v = *reinterpret_cast<const uint4 *>(src + ch * 16);
+    }
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    for (int j = 0; j < C; ++j) wts[rl * C + j] *= inv;
+  }
+  __syncthreads();
+  constexpr int kChunks = D / 8;  // 8 values (16 bytes of fp16) per work item
+  for (int t = threadIdx.x; got && t < nrows * kChunks; t += blockDim.x) {
+    const int rl = t / kChunks, ch = t % kChunks;
+    if (r0 + rl >= rows_here) continue;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < C; ++j) {
+      const float w = wts[rl * C + j];
+      if (w == 0.f) continue;
+      const uint4 v = *reinterpret_cast<const uint4 *>(rb + (j * rpc + rl) * M::kRowBytes + ch * 16);
       const __half2 *hv = reinterpret_cast<const __half2 *>(&v);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -320,14 +352,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         acc[2 * e + 1] += w * f.y;
       }
     }
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
     const int grow = row_base + r0 + rl;
     const int b = grow / sh.G, g = grow % sh.G;
     uint4 outv;
     uint32_t *po = reinterpret_cast<uint32_t *>(&outv);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      __nv_bfloat162 bv = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+      __nv_bfloat162 bv = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
       po[e] = *reinterpret_cast<uint32_t *>(&bv);
     }
     *reinterpret_cast<uint4 *>(a.o_out + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D +
@@ -341,23 +372,21 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   if (threadIdx.x == 0) DSA_TRACE_EVENT(11);
 }
 
-// Clusters of `cs` CTAs that can be resident at once with this kernel's shared
-// memory (index log2(cs)), queried once per device.
+// Clusters of each size (1..kMaxCluster) that can be resident at once with this
+// kernel, queried once per device.
 template <auto K>
 const int *active_clusters(size_t smem) {
-  static int cached[64][5];
+  static int cached[64][kMaxCluster + 1];
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
   if (!done[dev]) {
-    for (int lg = 0; lg <= 4; ++lg) {
-      const int cs = 1 << lg;
-      cached[dev][lg] = 0;
-      if (cs > 8 &&
-          cudaFuncSetAttribute(K, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-        cudaGetLastError();
-        continue;
-      }
+    const bool big =
+        cudaFuncSetAttribute(K, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+    cudaGetLastError();
+    for (int cs = 0; cs <= kMaxCluster; ++cs) {
+      cached[dev][cs] = 0;
+      if (cs == 0 || (cs > 8 && !big)) continue;
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(cs, 1, 1);
       cfg.blockDim = dim3(tc::kThreads, 1, 1);
@@ -370,7 +399,7 @@ const int *active_clusters(size_t smem) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, K, &cfg) == cudaSuccess) cached[dev][lg] = n;
+      if (cudaOccupancyMaxActiveClusters(&n, K, &cfg) == cudaSuccess) cached[dev][cs] = n;
       cudaGetLastError();
     }
     done[dev] = true;
@@ -378,19 +407,23 @@ const int *active_clusters(size_t smem) {
   return cached[dev];
 }
 
-// Cluster size for `nclusters` clusters sharing `kmax` pages each: the size with
-// the smallest (waves x pages per CTA), larger clusters on ties.
-inline int choose_cluster(const int *active, int nclusters, int kmax, int cap) {
+// Page CTAs per cluster for `nclusters` clusters sharing `kmax` pages each (one
+// more CTA takes the block's own tokens): the count with the smallest
+// (waves x tiles of the busiest CTA), more CTAs on ties.
+inline int choose_page_ctas(const int *active, int nclusters, int kmax, int page, int blk_tiles) {
   int best = 1;
   long long best_cost = -1;
-  for (int lg = 4; lg >= 0; --lg) {
-    const int cs = 1 << lg;
-    if (cs > cap || active[lg] < 1) continue;
-    const long long waves = (nclusters + active[lg] - 1) / active[lg];
-    const long long cost = waves * ((kmax + cs - 1) / cs + 1);  // +1: fixed per-CTA cost
+  for (int cp = kMaxCluster - 1; cp >= 1; --cp) {
+    const int cs = cp + 1;
+    if (active[cs] < 1) continue;
+    const int ppc = (kmax + cp - 1) / cp;
+    if (cp > 1 && (long long)(cp - 1) * ppc >= kmax) continue;  // a page CTA would be idle
+    const long long tiles = std::max((ppc * page + tc::kBN - 1) / tc::kBN, blk_tiles);
+    const long long waves = (nclusters + active[cs] - 1) / active[cs];
+    const long long cost = waves * (tiles + 1);  // +1: fixed per-CTA cost
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
-      best = cs;
+      best = cp;
     }
   }
   return best;
@@ -399,25 +432,27 @@ inline int choose_cluster(const int *active, int nclusters, int kmax, int cap) {
 template <int D, int PAGE>
 cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan_in, const SparseArgs &a,
                          cudaStream_t stream) {
+  using M = MergeLayout<D>;
   constexpr auto kern = sparse_attn<D, PAGE>;
   constexpr size_t kMaxSmem = 227 * 1024;
   cudaError_t err = set_smem_once<kern>(kMaxSmem);
   if (err != cudaSuccess) return err;
   SparsePlan plan = plan_in;
-  const int cs = choose_cluster(active_clusters<kern>(MergeLayout<D>::template kSmem<kSpStages>(
-                                    (sh.kmax + plan.cluster - 1) / plan.cluster)),
-                                sh.Hkv * sh.S * plan.rowtiles, sh.kmax, plan.cluster);
-  plan.cluster = cs;
-  plan.ppc = (sh.kmax + cs - 1) / cs;
-  const size_t smem = MergeLayout<D>::template kSmem<kSpStages>(plan.ppc);
+  const int *active = active_clusters<kern>(M::smem(kMaxCluster, std::max(sh.kmax, 64)));
+  const int cp = choose_page_ctas(active, sh.Hkv * sh.S * plan.rowtiles, sh.kmax, PAGE, plan.blk_tiles);
+  plan.cluster = cp + 1;
+  plan.ppc = (sh.kmax + cp - 1) / cp;
+  const size_t smem = M::smem(plan.cluster, plan.ppc);
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
   CUtensorMap kmap, vmap, kmap4, vmap4, bkmap, bvmap;
   const long long rows = sh.n_phys * sh.Hkv * PAGE;
   if ((err = make_kv_tensor_map(&kmap, a.k, rows, D, PAGE)) != cudaSuccess) return err;
   if ((err = make_kv_tensor_map(&vmap, a.v, rows, D, PAGE)) != cudaSuccess) return err;
-  if ((err = make_kv_pages_tensor_map(&kmap4, a.k, sh.n_phys, sh.Hkv, PAGE, D, tc::kBN / PAGE)) != cudaSuccess)
+  if ((err = make_kv_pages_tensor_map(&kmap4, a.k, sh.n_phys, sh.Hkv, PAGE, D, tc::kBN / PAGE)) !=
+      cudaSuccess)
     return err;
-  if ((err = make_kv_pages_tensor_map(&vmap4, a.v, sh.n_phys, sh.Hkv, PAGE, D, tc::kBN / PAGE)) != cudaSuccess)
+  if ((err = make_kv_pages_tensor_map(&vmap4, a.v, sh.n_phys, sh.Hkv, PAGE, D, tc::kBN / PAGE)) !=
+      cudaSuccess)
     return err;
   if ((err = make_blk_tensor_map(&bkmap, a.blk_k, (long long)sh.S * sh.B, sh.Hkv, D)) != cudaSuccess)
     return err;
@@ -448,10 +483,8 @@ DSA_TRACE_EXPORT(dsa_trace_sparse)
 SparsePlan plan_sparse(const Shape &sh, int /*num_sms*/) {
   SparsePlan p{};
   p.rowtiles = (sh.BG + kRowsPerCta - 1) / kRowsPerCta;
-  int cs = std::min(16, std::max(1, sh.kmax));
-  while (cs & (cs - 1)) cs &= cs - 1;  // power of two
-  p.cluster = cs;
-  p.ppc = (sh.kmax + cs - 1) / cs;
+  p.cluster = kMaxCluster;  // refined at launch from the device's cluster capacity
+  p.ppc = (sh.kmax + kMaxCluster - 2) / (kMaxCluster - 1);
   p.blk_tiles = (sh.B + tc::kBN - 1) / tc::kBN;
   p.total = 4096;  // status word only: partials never leave the cluster
   return p;

@@ -160,8 +160,8 @@ struct Engine {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // (a policy whose tile addresses come from a table built in prepare()
-    // issues its first loads once that table is complete)
+    pol.ready();  // tables built by prepare() are complete from here on
+    // (a policy whose first tile addresses need those tables issues them now)
     if (!Policy::kIssueBeforeSync && threadIdx.x == 0 && num_tiles > 0) issue_first(pol, num_tiles);
     tmem = *reinterpret_cast<volatile uint32_t *>(smem + L::kOffMisc);
     ctx = sm100::WaitCtx{abort_flag(), status};
