@@ -43,6 +43,8 @@ WORKLOAD_TEXT = {
             "selection of block n+1 on a second stream overlapped with block n's sparse steps",
     "8k": "8k: 1 seq, N=8192, B=32, Hq=32, Hkv=8, d=128, page=16, top-k 512 tokens, 32 steps",
     "32k": "32k: 1 seq, N=32768, B=32, Hq=28, Hkv=4, d=128, page=64, top-k 1024 tokens, 32 steps",
+    "tiny": "tiny: 1 seq, N=1024, B=4, Hq=4, Hkv=1, d=64, page=16, top-k 128 tokens, 4 steps, "
+            "8 planted needle pages",
     "batched": "batched: 8 seqs, N~U[16K,64K], B=32, Hq=32, Hkv=8, d=128, page=16, "
                "top-k in {512,1024,2048}, 32 steps, random page table",
 }
@@ -156,15 +158,21 @@ class ClockSampler:
                 "samples": len(self.rows)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU (torch.distributed.run sets RANK/LOCAL_RANK/WORLD_SIZE).
+    The process group carries only the barrier and the max-over-ranks time; the
+    "gloo" backend serves the CPU tests of this plumbing."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
     elif n_gpus > 1:
         raise SystemExit("--gpus N > 1 must be launched with torch.distributed.run")
     return world, rank, local
@@ -180,7 +188,8 @@ def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
