@@ -64,6 +64,33 @@ T *at(void *ws, size_t off) {
 
 }  // namespace
 
+// Scratch of dsa_select_static_scratch, for callers that may not allocate (a
+// runtime plugin handed only its inputs and outputs, a path running while the
+// memory pool is fully reserved).  The CUDA module sets it aside on each device
+// when it is loaded; no allocation call is involved.  One array per device, so
+// calls on one device must not overlap in time.
+static __device__ __align__(256) unsigned char select_static_scratch[DSA_SELECT_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of select_static_scratch on the current device, looked up once
+// per device (the lookup may load the module, hence: first call outside capture).
+void *static_scratch_current() {
+  static void *cache[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, select_static_scratch) != cudaSuccess) return nullptr;
+    cache[dev] = p;
+  }
+  return cache[dev];
+}
+
+}  // namespace
+
 extern "C" {
 
 int dsa_version(void) { return 100; }
@@ -84,6 +111,9 @@ const char *dsa_strerror(int code) {
     case DSA_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
     case DSA_ERR_BAD_INDEX: return "page index or page-table entry out of range";
     case DSA_ERR_NONFINITE: return "non-finite page score (non-finite inputs)";
+    case DSA_ERR_SCRATCH_LIMIT:
+      return "shape needs more scratch than the 16 MiB static array of dsa_select_static_scratch "
+             "(use dsa_select with a caller workspace)";
     default: return "unknown status code";
   }
 }
@@ -154,6 +184,44 @@ int dsa_select(const void *q_blk, const void *k_cache, const void *v_cache,
   a.mtile = at<float>(workspace, plan.off_mtile);
   a.scores = at<float>(workspace, plan.off_scores);
   a.status = at<uint32_t>(workspace, 0);
+  if (dsa::launch_select(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+int dsa_select_static_scratch(const void *q_blk, const void *k_cache, const void *v_cache,
+                              const int32_t *n_ctx, int32_t page, const int32_t *topk,
+                              int32_t *idx_out, void *o_out, dsa_stream_t stream,
+                              const dsa_dims *dims, int32_t *cnt_out, uint32_t *status) {
+  Shape sh;
+  int rc = make_shape(dims, &sh);
+  if (rc != DSA_OK) return rc;
+  if (page != sh.P) return DSA_ERR_INVALID_ARG;
+  if (!q_blk || !k_cache || !v_cache || !n_ctx || !topk || !idx_out || !o_out || !cnt_out ||
+      !status)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o_out) ||
+      (reinterpret_cast<uintptr_t>(status) & 3u) != 0)
+    return DSA_ERR_INVALID_ARG;
+  const dsa::SelectPlan plan = dsa::plan_select(sh, num_sms_current());
+  if (plan.total > DSA_SELECT_STATIC_SCRATCH_BYTES) return DSA_ERR_SCRATCH_LIMIT;
+  void *scratch = static_scratch_current();
+  if (scratch == nullptr) return DSA_ERR_CUDA;
+  dsa::SelectArgs a{};
+  a.q = static_cast<const __nv_bfloat16 *>(q_blk);
+  a.k = static_cast<const __nv_bfloat16 *>(k_cache);
+  a.v = static_cast<const __nv_bfloat16 *>(v_cache);
+  a.n_ctx = n_ctx;
+  a.topk = topk;
+  a.idx_out = idx_out;
+  a.cnt_out = cnt_out;
+  a.o_out = static_cast<__nv_bfloat16 *>(o_out);
+  a.part_o = at<float>(scratch, plan.off_part_o);
+  a.part_ml = at<float>(scratch, plan.off_part_ml);
+  a.pagepart = at<float>(scratch, plan.off_pagepart);
+  a.mtile = at<float>(scratch, plan.off_mtile);
+  a.scores = at<float>(scratch, plan.off_scores);
+  a.status = status;  // the caller's word; the array's header bytes stay unused
   if (dsa::launch_select(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;

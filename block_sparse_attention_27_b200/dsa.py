@@ -23,11 +23,15 @@ DSA_ERR_CUDA = -4
 DSA_ERR_DEVICE_TIMEOUT = -5
 DSA_ERR_BAD_INDEX = -6
 DSA_ERR_NONFINITE = -7
+DSA_ERR_SCRATCH_LIMIT = -8
+
+# size of the library-held scratch array of dsa_select_static_scratch
+DSA_SELECT_STATIC_SCRATCH_BYTES = 16 << 20
 
 # every symbol include/dsa.h declares
 EXPORTED = ("dsa_select", "dsa_sparse_attn", "dsa_select_workspace_size",
             "dsa_sparse_workspace_size", "dsa_workspace_init", "dsa_get_status",
-            "dsa_strerror", "dsa_kernels_per_call", "dsa_version")
+            "dsa_strerror", "dsa_kernels_per_call", "dsa_version", "dsa_select_static_scratch")
 
 
 class DsaError(RuntimeError):
@@ -59,6 +63,9 @@ def load(path: str = LIB_PATH):
     dims_p = ctypes.POINTER(dsa_dims)
     lib.dsa_select.restype = ci
     lib.dsa_select.argtypes = [vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, dims_p, vp, vp, sz]
+    lib.dsa_select_static_scratch.restype = ci
+    lib.dsa_select_static_scratch.argtypes = [vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp,
+                                              dims_p, vp, vp]
     lib.dsa_sparse_attn.restype = ci
     lib.dsa_sparse_attn.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, dims_p, vp, vp, vp, sz]
     lib.dsa_select_workspace_size.restype = sz
@@ -159,6 +166,33 @@ def dsa_select(q_blk, k_cache, v_cache, n_ctx, page, topk, idx_out, o_out, strea
                            ctypes.byref(dims), _ptr(cnt_out), _ptr(workspace.buf), workspace.nbytes)
     if rc != DSA_OK:
         raise DsaError(rc, "dsa_select")
+
+
+def dsa_select_static_scratch(q_blk, k_cache, v_cache, n_ctx, page, topk, idx_out, o_out,
+                              stream=None, *, dims: dsa_dims, cnt_out, status):
+    """Selection pass with the library's static scratch instead of a workspace (see
+    include/dsa.h).  `status` is a device int32/uint32 tensor of one element that
+    holds 0 before the first call; read it with status_word().  Raises DsaError."""
+    _check(q_blk, "q_blk", torch.bfloat16, 4)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(n_ctx, "n_ctx", torch.int32)
+    _check(topk, "topk", torch.int32)
+    _check(idx_out, "idx_out", torch.int32)
+    _check(o_out, "o_out", torch.bfloat16)
+    _check(cnt_out, "cnt_out", torch.int32)
+    _check(status, "status", torch.int32)
+    rc = load().dsa_select_static_scratch(_ptr(q_blk), _ptr(k_cache), _ptr(v_cache), _ptr(n_ctx),
+                                          int(page), _ptr(topk), _ptr(idx_out), _ptr(o_out),
+                                          _stream(stream), ctypes.byref(dims), _ptr(cnt_out),
+                                          _ptr(status))
+    if rc != DSA_OK:
+        raise DsaError(rc, "dsa_select_static_scratch")
+
+
+def status_word(status, stream=None) -> int:
+    """dsa_get_status() of a caller-owned status word (synchronises `stream`)."""
+    return int(load().dsa_get_status(_ptr(status), _stream(stream)))
 
 
 def dsa_sparse_attn(q_blk, k_cache, v_cache, idx, blk_k, blk_v, o_out, stream=None, *,

@@ -15,7 +15,8 @@
  *  Element types: q/k/v/blk_k/blk_v/o are bf16 (2-byte IEEE bfloat16); index
  *  arrays are int32.  Every pointer passed here is a DEVICE pointer unless the
  *  argument says "host".  The caller owns all memory; the library allocates
- *  nothing and keeps no state except a per-device cache of the SM count.
+ *  nothing and keeps no state except a per-device cache of the SM count (and the
+ *  fixed scratch array of dsa_select_static_scratch, see there).
  *
  *  Layouts (row-major, innermost last):
  *    q_blk        [S, B, Hq, d]          queries of the block (post-RoPE)
@@ -72,6 +73,10 @@ extern "C" {
 #define DSA_ERR_DEVICE_TIMEOUT (-5)     /* a bounded device wait gave up */
 #define DSA_ERR_BAD_INDEX (-6)          /* idx entry >= number of pages, or page-table entry outside the cache */
 #define DSA_ERR_NONFINITE (-7)          /* a page score was NaN or Inf (non-finite inputs) */
+#define DSA_ERR_SCRATCH_LIMIT (-8)      /* shape needs more than DSA_SELECT_STATIC_SCRATCH_BYTES (dsa_select_static_scratch only) */
+
+/* Size of the library-held scratch array used by dsa_select_static_scratch. */
+#define DSA_SELECT_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 
 typedef struct dsa_dims {
   int32_t S;          /* sequences in the batch */
@@ -140,6 +145,52 @@ int dsa_workspace_init(void *workspace, size_t ws_bytes, dsa_stream_t stream);
  * the most severe device-side code recorded since dsa_workspace_init(); the word
  * is left as it is (sticky).  Returns DSA_ERR_CUDA if the read fails. */
 int dsa_get_status(const void *workspace, dsa_stream_t stream);
+
+/*
+ * Selection pass without a workspace.  The MAGE page has no counterpart of this
+ * entry point: it serves deployment, not the method.
+ *
+ * Who needs it: a caller that is handed only its inputs and outputs and may not
+ * allocate device memory at this point (for instance a plugin of an inference
+ * runtime whose host hands it no workspace, or a path that runs while the
+ * process's memory pool is fully reserved) cannot supply the workspace
+ * dsa_select needs.  This variant launches the same three kernels as dsa_select
+ * with their scratch placed in a fixed device array that the library itself
+ * holds: a file-scope __device__ array of DSA_SELECT_STATIC_SCRATCH_BYTES
+ * (16 MiB) per device, set aside when the CUDA module is loaded, not by an
+ * allocation call.  The call allocates nothing.
+ *
+ * Limit: the shape's dsa_select_workspace_size() must not exceed
+ * DSA_SELECT_STATIC_SCRATCH_BYTES; a larger shape returns DSA_ERR_SCRATCH_LIMIT
+ * before anything is launched (use dsa_select with a caller workspace).  On a
+ * 148-SM B200 this admits an 8K prefix with 8 KV heads, 32 query tokens,
+ * d = 128, page 16 (10.6 MiB) and a 32K prefix with 4 KV heads, page 64
+ * (13.3 MiB), not a 128K prefix with 8 KV heads (49 MiB).
+ *
+ * Arguments: those of dsa_select without workspace/ws_bytes, plus
+ *   status: device uint32, caller-owned, 4-byte aligned, receiving the device
+ *   status bits.  It must hold 0 before the first call; the kernels only OR bits
+ *   into it (sticky, like the workspace status word).  dsa_get_status(status,
+ *   stream) reads it (it only reads the first word of what it is given); writing
+ *   0 clears it.
+ * The scratch array needs no zeroing: every word of it a call reads was written
+ * earlier in the same call.
+ *
+ * Concurrency: the scratch array is one per device, shared by every call on that
+ * device.  Calls on one device must not overlap in time: issue them on one
+ * stream or order them with events.  Two calls in flight together on different
+ * streams of one device race on the scratch and return wrong results without
+ * any error.  Calls on different devices are independent.
+ *
+ * First call on a device: the array's address is looked up
+ * (cudaGetSymbolAddress, with that device current) and cached per device.  The
+ * lookup may load the library's CUDA module, so make the first call on each
+ * device outside stream capture.
+ */
+int dsa_select_static_scratch(const void *q_blk, const void *k_cache, const void *v_cache,
+                              const int32_t *n_ctx, int32_t page, const int32_t *topk,
+                              int32_t *idx_out, void *o_out, dsa_stream_t stream,
+                              const dsa_dims *dims, int32_t *cnt_out, uint32_t *status);
 
 /* Static description of a status code. */
 const char *dsa_strerror(int code);

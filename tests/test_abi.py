@@ -101,3 +101,22 @@ def test_library_has_no_oracle_dependency():
     for py in ("dsa.py", "build.py", "__init__.py"):
         text = open(os.path.join(B.PKG, py)).read()
         assert "import oracle" not in text and "from oracle" not in text
+
+
+def test_static_scratch_entry_checks_on_host(lib):
+    """dsa_select_static_scratch: arguments checked like dsa_select, a status word is
+    required, and shapes beyond the static array are refused before any launch."""
+    ok = ctypes.c_void_p(1 << 20)
+    dims = good_dims()
+    rc = lib.dsa_select_static_scratch(ok, ok, ok, ok, 16, ok, ok, ok, None, ctypes.byref(dims),
+                                       ok, None)
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+    rc = lib.dsa_select_static_scratch(ok, ok, ok, ok, 16, ok, ok, ok, None, ctypes.byref(dims),
+                                       ok, ctypes.c_void_p((1 << 20) + 2))
+    assert rc == dsa.DSA_ERR_INVALID_ARG
+    big = good_dims(max_pages=8192, n_phys=8192, kmax=64)      # 128K prefix, 8 KV heads
+    assert lib.dsa_select_workspace_size(ctypes.byref(big)) > dsa.DSA_SELECT_STATIC_SCRATCH_BYTES
+    rc = lib.dsa_select_static_scratch(ok, ok, ok, ok, 16, ok, ok, ok, None, ctypes.byref(big),
+                                       ok, ok)
+    assert rc == dsa.DSA_ERR_SCRATCH_LIMIT
+    assert "static" in dsa.strerror(dsa.DSA_ERR_SCRATCH_LIMIT)
