@@ -15,6 +15,8 @@
 //   3. select_topk: radix select of the kp-th largest score per (seq, KV head),
 //      ties broken towards the lower page index, emitted in ascending order.
 #include <algorithm>
+#include <cstring>
+#include <type_traits>
 
 #include "launch.h"
 #include "sm100.cuh"
@@ -153,19 +155,24 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const SelectArgs &a = pp.a;
   const int s = blockIdx.z, h = blockIdx.y;
   const int split = blockIdx.x / plan.rowtiles, rt = blockIdx.x % plan.rowtiles;
-  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status,
-                             threadIdx.x == 0 && blockIdx.x == 0);
-  const int ntiles = (n + tc::kBN - 1) / tc::kBN;
-  const int t_begin = split * plan.tiles_per_split;
-  const int num_tiles = max(0, min(ntiles, t_begin + plan.tiles_per_split) - t_begin);
-
   if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
-  const size_t sh_idx = (size_t)s * sh.Hkv + h;
   SelectPolicy<D, PAGE> pol;
   pol.kmap = &kmap;
   pol.vmap = &vmap;
   pol.kmap4 = &kmap4;
   pol.vmap4 = &vmap4;
+  tc::Engine<D, kSelStages> eng;
+  eng.setup(smem_raw, pol);
+  // everything below may read what the kernel ahead of this one wrote
+  sm100::grid_dep_wait();
+  sm100::grid_dep_launch_dependents();
+
+  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status,
+                             threadIdx.x == 0 && blockIdx.x == 0);
+  const int ntiles = (n + tc::kBN - 1) / tc::kBN;
+  const int t_begin = split * plan.tiles_per_split;
+  const int num_tiles = max(0, min(ntiles, t_begin + plan.tiles_per_split) - t_begin);
+  const size_t sh_idx = (size_t)s * sh.Hkv + h;
   pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
   pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
   pol.mtile_head = a.mtile + sh_idx * plan.max_tiles * sh.BG;
@@ -183,8 +190,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.t_begin = t_begin;
   pol.row_base = rt * kRowsPerCta;
   pol.sl2 = sh.sl2;
-  tc::Engine<D, kSelStages> eng;
-  eng.init(smem_raw, a.status, pol, num_tiles);
+  eng.init(a.status, pol, num_tiles);
   float m, l;
   eng.template run<PAGE>(pol, num_tiles, m, l);
   float m_row, l_row, wa, wb;
@@ -232,27 +238,147 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // output CTAs write o_out = sum_j 2^(m_j - M) O_j / L in bf16.
 // ---------------------------------------------------------------------------
 constexpr int kFinThreads = 256;
-constexpr int kRowsPerFinCta = 8;
+constexpr int kRowsPerFinCta = 8;   // output CTAs: one query row per warp
+constexpr int kFinTiles = 2;        // score CTAs: 64-token tiles a warp loads at once
+constexpr int kFinBatch = 16;       // output CTAs: split partials a lane loads at once
 
+// Folds a partial (m, l) into the running (M, L) of a row (log2 domain); an
+// empty partial (l = 0) leaves it unchanged.
+__device__ __forceinline__ void merge_ml(float &M, float &L, float m, float l) {
+  if (!(l > 0.f)) return;
+  if (m > M) {
+    L = L * exp2f(M - m) + l;
+    M = m;
+  } else {
+    L += l * exp2f(m - M);
+  }
+}
+
+// sM[row] = M and sLinv[row] = 1/L over all splits.  Each row gets tpr = the
+// largest power of two <= blockDim.x / BG (at most 32) threads of one warp; each
+// of them loads its splits 8 at a time (all in flight together), then the tpr
+// partial results are combined with shuffles.
 __device__ __forceinline__ void merged_row_stats(const Shape &sh, const SelectPlan &plan,
                                                  const float *part_ml, size_t sh_idx, float *sM,
                                                  float *sLinv) {
-  for (int row = threadIdx.x; row < sh.BG; row += blockDim.x) {
+  int tpr = 1;
+  while (tpr < 32 && 2 * tpr * sh.BG <= (int)blockDim.x) tpr *= 2;
+  const int sub = threadIdx.x % tpr;
+  const int per_pass = (int)blockDim.x / tpr;
+  const float2 *ml = reinterpret_cast<const float2 *>(part_ml) + sh_idx * plan.splits * sh.BG;
+  // every thread runs the same passes (the shuffles need whole warps)
+  for (int row0 = 0; row0 < sh.BG; row0 += per_pass) {
+    const int row = row0 + (int)threadIdx.x / tpr;
+    const bool valid = row < sh.BG;
     float M = -INFINITY, L = 0.f;
-#pragma unroll 4
-    for (int j = 0; j < plan.splits; ++j) {
-      const float2 ml = *reinterpret_cast<const float2 *>(
-          part_ml + ((sh_idx * plan.splits + j) * sh.BG + row) * 2);
-      if (!(ml.y > 0.f)) continue;
-      if (ml.x > M) {
-        L = L * exp2f(M - ml.x) + ml.y;
-        M = ml.x;
-      } else {
-        L += ml.y * exp2f(ml.x - M);
+    for (int j0 = sub; j0 < plan.splits; j0 += 8 * tpr) {
+      float2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * tpr;
+        v[u] = (valid && j < plan.splits) ? ml[(size_t)j * sh.BG + row] : make_float2(-INFINITY, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) merge_ml(M, L, v[u].x, v[u].y);
+    }
+    for (int o = tpr / 2; o > 0; o >>= 1) {
+      const float M2 = __shfl_xor_sync(0xffffffffu, M, o);
+      const float L2 = __shfl_xor_sync(0xffffffffu, L, o);
+      merge_ml(M, L, M2, L2);
+    }
+    if (valid && sub == 0) {
+      sM[row] = M;
+      sLinv[row] = L > 0.f ? 1.f / L : 0.f;
+    }
+  }
+}
+
+// Page scores of the pages [p0, p1) (tile-aligned) of one (sequence, KV head).
+// Lane i of a warp handles the rows VEC*i + 32*VEC*c (c < kChunks): their M and
+// 1/L stay in registers, and for kFinTiles tiles at a time the tile maxima and
+// every unit's partial masses are loaded before any of them is used.
+template <int PAGE, int VEC, int kChunks>
+__device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &plan,
+                                            const SelectArgs &a, size_t sh_idx, int np, int p0,
+                                            int p1, const float *sM, const float *sLinv) {
+  using U = tc::Units<PAGE>;
+  using V = typename std::conditional<VEC == 4, float4, float>::type;
+  constexpr int kPagesPerTile = tc::kBN / PAGE;
+  constexpr int kUnitsPerTile = U::kPerTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int BG = sh.BG;
+  float rm[kChunks][VEC], rl[kChunks][VEC];
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const int row = VEC * lane + 32 * VEC * c + e;
+      rm[c][e] = row < BG ? sM[row] : 0.f;
+      rl[c][e] = row < BG ? sLinv[row] : 0.f;  // 0: the row does not exist
+    }
+  auto load = [&](const float *base, int c) -> V {
+    const int row = VEC * lane + 32 * VEC * c;
+    if (row >= BG) {
+      V z;
+      memset(&z, 0, sizeof z);
+      return z;
+    }
+    return *reinterpret_cast<const V *>(base + row);
+  };
+  auto lanes = [](const V &v, int e) -> float { return reinterpret_cast<const float *>(&v)[e]; };
+  const float inv_bg = 1.f / (float)BG;
+  const int warps = (int)blockDim.x / 32;
+  const float *mt_head = a.mtile + sh_idx * plan.max_tiles * BG;
+  const float *pp_head = a.pagepart + sh_idx * sh.max_pages * U::kPerPage * BG;
+  for (int lp0 = p0 + warp * kPagesPerTile * kFinTiles; lp0 < p1;
+       lp0 += warps * kPagesPerTile * kFinTiles) {
+    V mt[kFinTiles][kChunks];
+    V part[kFinTiles][kUnitsPerTile][kChunks];
+#pragma unroll
+    for (int t = 0; t < kFinTiles; ++t) {
+      const int lpt = lp0 + t * kPagesPerTile;
+      const bool live = lpt < min(np, p1);
+      const int tile = lpt * PAGE / tc::kBN;
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        if (live) {
+          mt[t][c] = load(mt_head + (size_t)tile * BG, c);
+        } else {
+          memset(&mt[t][c], 0, sizeof(V));
+        }
+#pragma unroll
+        for (int u = 0; u < kUnitsPerTile; ++u) {
+          if (live && lpt + u / U::kPerPage < np) {
+            part[t][u][c] = load(pp_head + ((size_t)lpt * U::kPerPage + u) * BG, c);
+          } else {
+            memset(&part[t][u][c], 0, sizeof(V));
+          }
+        }
       }
     }
-    sM[row] = M;
-    sLinv[row] = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int t = 0; t < kFinTiles; ++t) {
+      const int lpt = lp0 + t * kPagesPerTile;
+      float acc[kUnitsPerTile];
+#pragma unroll
+      for (int u = 0; u < kUnitsPerTile; ++u) acc[u] = 0.f;
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          const float f = rl[c][e] > 0.f ? exp2f(lanes(mt[t][c], e) - rm[c][e]) * rl[c][e] : 0.f;
+#pragma unroll
+          for (int u = 0; u < kUnitsPerTile; ++u) acc[u] += lanes(part[t][u][c], e) * f;
+        }
+#pragma unroll
+      for (int pi = 0; pi < kPagesPerTile; ++pi) {
+        float v = 0.f;
+#pragma unroll
+        for (int u = pi * U::kPerPage; u < (pi + 1) * U::kPerPage; ++u) v += acc[u];
+        v = warp_sum(v) * inv_bg;
+        if (lane == 0 && lpt + pi < p1) a.scores[sh_idx * sh.max_pages + lpt + pi] = v;
+      }
+    }
   }
 }
 
@@ -262,6 +388,8 @@ __global__ void __launch_bounds__(kFinThreads) select_finalize(const __grid_cons
   const Shape &sh = pp.sh;
   const SelectPlan &plan = pp.plan;
   const SelectArgs &a = pp.a;
+  sm100::grid_dep_wait();  // the partials of select_partial
+  sm100::grid_dep_launch_dependents();
   const int s = blockIdx.z, h = blockIdx.y;
   const size_t sh_idx = (size_t)s * sh.Hkv + h;
   const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status, false);
@@ -271,55 +399,59 @@ __global__ void __launch_bounds__(kFinThreads) select_finalize(const __grid_cons
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int score_ctas = (sh.max_pages + plan.fin_pages - 1) / plan.fin_pages;
   if ((int)blockIdx.x < score_ctas) {
-    // a warp takes one 64-token tile (64/PAGE pages) at a time: the row factor
-    // 2^(mtile - M) / L is shared by the tile's pages, and all loads of the tile
-    // are in flight together before the per-page warp reductions
-    using U = tc::Units<PAGE>;
-    constexpr int kPagesPerTile = tc::kBN / PAGE;
-    constexpr int kUnitsPerTile = tc::kBN / U::kKeys;
-    const float inv_bg = 1.f / (float)sh.BG;
     const int p0 = blockIdx.x * plan.fin_pages;  // a multiple of 64 tokens
     const int p1 = min(sh.max_pages, p0 + plan.fin_pages);
-    for (int lp0 = p0 + warp * kPagesPerTile; lp0 < p1; lp0 += (kFinThreads / 32) * kPagesPerTile) {
-      const int tile = lp0 * PAGE / tc::kBN;
-      float acc[kUnitsPerTile];
-#pragma unroll
-      for (int u = 0; u < kUnitsPerTile; ++u) acc[u] = 0.f;
-      if (lp0 < np) {
-        const float *mt = a.mtile + (sh_idx * plan.max_tiles + tile) * sh.BG;
-        const float *part = a.pagepart + (sh_idx * sh.max_pages + lp0) * U::kPerPage * sh.BG;
-        for (int row = lane; row < sh.BG; row += 32) {
-          const float f = exp2f(mt[row] - sM[row]) * sLinv[row];
-#pragma unroll
-          for (int u = 0; u < kUnitsPerTile; ++u)
-            if (lp0 + u / U::kPerPage < np) acc[u] += part[(size_t)u * sh.BG + row] * f;
-        }
-      }
-#pragma unroll
-      for (int pi = 0; pi < kPagesPerTile; ++pi) {
-        float v = 0.f;
-#pragma unroll
-        for (int u = pi * U::kPerPage; u < (pi + 1) * U::kPerPage; ++u) v += acc[u];
-        v = warp_sum(v) * inv_bg;
-        if (lane == 0 && lp0 + pi < p1) a.scores[sh_idx * sh.max_pages + lp0 + pi] = v;
-      }
+    if (sh.BG % 4 == 0) {
+      if (sh.BG <= 128) page_scores<PAGE, 4, 1>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
+      else page_scores<PAGE, 4, 2>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
+    } else {
+      if (sh.BG <= 32) page_scores<PAGE, 1, 1>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
+      else page_scores<PAGE, 1, 8>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
     }
   } else {
+    // o_out row: lane j holds the weight 2^(m_j - M) of split j (0 for an empty
+    // split, whose O was never written); kFinBatch splits' O loads are in flight
+    // together
     const int row = (blockIdx.x - score_ctas) * kRowsPerFinCta + warp;
     if (row >= sh.BG) return;
     const int b = row / sh.G, g = row % sh.G;
+    static_assert(D / 32 == 4 || D / 32 == 2, "columns per lane");
     constexpr int kPer = D / 32;
+    using V = typename std::conditional<kPer == 4, float4, float2>::type;
     float acc[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
-    for (int j = 0; j < plan.splits; ++j) {
-      const size_t r = (sh_idx * plan.splits + j) * sh.BG + row;
-      const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + r * 2);
-      if (!(ml.y > 0.f)) continue;
-      const float w = exp2f(ml.x - sM[row]);
-      const float *src = a.part_o + r * D + lane * kPer;
+    const float Mrow = sM[row];
+    for (int j0 = 0; j0 < plan.splits; j0 += 32) {
+      float w_lane = 0.f;
+      if (j0 + lane < plan.splits) {
+        const size_t r = (sh_idx * plan.splits + j0 + lane) * sh.BG + row;
+        const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + r * 2);
+        w_lane = ml.y > 0.f ? exp2f(ml.x - Mrow) : 0.f;
+      }
+      const int nj = min(32, plan.splits - j0);
+      for (int jb = 0; jb < nj; jb += kFinBatch) {
+        V o[kFinBatch];
+        float w[kFinBatch];
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) acc[i] += w * src[i];
+        for (int u = 0; u < kFinBatch; ++u) {
+          w[u] = __shfl_sync(0xffffffffu, w_lane, (jb + u) & 31);
+          const bool use = jb + u < nj && w[u] > 0.f;
+          if (use) {
+            const size_t r = (sh_idx * plan.splits + j0 + jb + u) * sh.BG + row;
+            o[u] = *reinterpret_cast<const V *>(a.part_o + r * D + lane * kPer);
+          } else {
+            memset(&o[u], 0, sizeof(V));
+            w[u] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kFinBatch; ++u) {
+          const float *ov = reinterpret_cast<const float *>(&o[u]);
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) acc[i] += w[u] * ov[i];
+        }
+      }
     }
     __nv_bfloat16 *dst = a.o_out + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D + lane * kPer;
 #pragma unroll
@@ -352,6 +484,8 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk(const __grid_constan
   __shared__ int s_bad;
   const Shape &sh = pp.sh;
   const SelectArgs &a = pp.a;
+  sm100::grid_dep_wait();  // the page scores of select_finalize
+  sm100::grid_dep_launch_dependents();
   const int s = blockIdx.y, h = blockIdx.x;
   const size_t sh_idx = (size_t)s * sh.Hkv + h;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -505,12 +639,31 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
   constexpr size_t smem = tc::Layout<D, kSelStages>::kAlloc;
   err = set_smem_once<kern>(smem);
   if (err != cudaSuccess) return err;
-  dim3 grid(plan.splits * plan.rowtiles, sh.Hkv, sh.S);
-  kern<<<grid, tc::kThreads, smem, stream>>>(pp, kmap, vmap, kmap4, vmap4);
+  // all three kernels are programmatic dependents of the kernel ahead of them:
+  // each one's set-up overlaps the tail of the previous one
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(plan.splits * plan.rowtiles, sh.Hkv, sh.S);
+  cfg.blockDim = dim3(tc::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  err = cudaLaunchKernelEx(&cfg, kern, pp, kmap, vmap, kmap4, vmap4);
+  if (err != cudaSuccess) return err;
   const int score_ctas = (sh.max_pages + plan.fin_pages - 1) / plan.fin_pages;
   const int o_ctas = (sh.BG + kRowsPerFinCta - 1) / kRowsPerFinCta;
-  select_finalize<D, PAGE><<<dim3(score_ctas + o_ctas, sh.Hkv, sh.S), kFinThreads, 0, stream>>>(pp);
-  select_topk<<<dim3(sh.Hkv, sh.S), kTopkThreads, 0, stream>>>(pp);
+  cfg.gridDim = dim3(score_ctas + o_ctas, sh.Hkv, sh.S);
+  cfg.blockDim = dim3(kFinThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  err = cudaLaunchKernelEx(&cfg, select_finalize<D, PAGE>, pp);
+  if (err != cudaSuccess) return err;
+  cfg.gridDim = dim3(sh.Hkv, sh.S, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  err = cudaLaunchKernelEx(&cfg, select_topk, pp);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

@@ -117,6 +117,19 @@ __device__ __forceinline__ void cluster_sync() {
                    : "memory");
 }
 // Split form: every thread arrives once (release) and later waits once (acquire).
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start while the kernel before it on the stream is still
+// running; grid_dep_wait() returns once that kernel has completed and its
+// memory is visible (at once if there is no such dependency), so nothing the
+// caller passes may be read before it.  grid_dep_launch_dependents() lets the
+// next such kernel on the stream start its own set-up.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }

@@ -196,21 +196,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const int h = blockIdx.y;
   const int s = blockIdx.z / plan.rowtiles, rt = blockIdx.z % plan.rowtiles;
   const size_t sh_idx = (size_t)s * sh.Hkv + h;
-  const bool reporter = threadIdx.x == 0 && c == 0 && rt == 0;
-  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status, reporter && h == 0);
-  int cnt = a.idx_cnt[sh_idx];
-  if (cnt < 0 || cnt > sh.kmax) {
-    if (reporter) raise_status(a.status, kStatusBadIndex);
-    cnt = max(0, min(cnt, sh.kmax));
-  }
-  // CTAs 0..C-2: pages; CTA C-1: the block's own tokens
-  const bool blk_cta = c == C - 1;
-  const int e_begin = blk_cta ? cnt : min(cnt, c * plan.ppc);
-  const int e_end = blk_cta ? cnt : min(cnt, (c + 1) * plan.ppc);
-  constexpr int kPagesPerTile = tc::kBN / PAGE;
-  const int sel_tiles = (e_end - e_begin + kPagesPerTile - 1) / kPagesPerTile;
-  const int num_tiles = sel_tiles + (blk_cta ? plan.blk_tiles : 0);
   const int row_base = rt * kRowsPerCta;
+  const bool blk_cta = c == C - 1;  // CTAs 0..C-2: pages; CTA C-1: the block's own tokens
+  constexpr int kPagesPerTile = tc::kBN / PAGE;
 
   SparsePolicy<D, PAGE> pol;
   pol.kmap = &kmap;
@@ -219,6 +207,25 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.vmap4 = &vmap4;
   pol.bkmap = &bkmap;
   pol.bvmap = &bvmap;
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
+  tc::Engine<D, kSpStages> eng;
+  eng.setup(smem_raw, pol);
+  // everything below may read what the kernel ahead of this one wrote
+  sm100::grid_dep_wait();
+  sm100::grid_dep_launch_dependents();
+
+  const bool reporter = threadIdx.x == 0 && c == 0 && rt == 0;
+  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status, reporter && h == 0);
+  int cnt = a.idx_cnt[sh_idx];
+  if (cnt < 0 || cnt > sh.kmax) {
+    if (reporter) raise_status(a.status, kStatusBadIndex);
+    cnt = max(0, min(cnt, sh.kmax));
+  }
+  const int e_begin = blk_cta ? cnt : min(cnt, c * plan.ppc);
+  const int e_end = blk_cta ? cnt : min(cnt, (c + 1) * plan.ppc);
+  const int sel_tiles = (e_end - e_begin + kPagesPerTile - 1) / kPagesPerTile;
+  const int num_tiles = sel_tiles + (blk_cta ? plan.blk_tiles : 0);
+
   pol.idx_row = a.idx + sh_idx * sh.kmax;
   pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
   pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
@@ -242,9 +249,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.sel_tiles = sel_tiles;
   pol.row_base = row_base;
   pol.sl2 = sh.sl2;
-  if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
-  tc::Engine<D, kSpStages> eng;
-  eng.init(smem_raw, a.status, pol, num_tiles);
+  eng.init(a.status, pol, num_tiles);
   // rows this CTA owns in the merge, and the bytes it will receive for them
   const int rpc = (int)M::rpc(C);
   const int r0 = c * rpc;
@@ -464,13 +469,16 @@ cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan_in, const Spars
   cfg.blockDim = dim3(tc::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = plan.cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // the set-up before grid_dep_wait() may overlap the kernel ahead on the stream
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   err = cudaLaunchKernelEx(&cfg, kern, prm, kmap, vmap, kmap4, vmap4, bkmap, bvmap);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();

@@ -103,35 +103,19 @@ struct Engine {
   __device__ __forceinline__ int group() const { return (warp - 2) >> 2; }  // softmax group 0 or 1
   __device__ __forceinline__ uint32_t lane_tmem() const { return tmem + ((uint32_t)(quarter() * 32) << 16); }
 
-  // Barrier init and TMEM allocation; every thread of the CTA calls it.  The
-  // softmax threads already copy their query rows into the Q tile, and (for a
-  // policy that allows it) the producer issues the loads of the first STAGES
-  // tiles, before the CTA-wide barrier.
+  // Set-up that reads no memory the caller passes: shared-memory carve-up,
+  // barrier init, tensor-map prefetch (thread 0) and the TMEM allocation (warp
+  // 1).  Every thread of the CTA calls it; a kernel launched as a programmatic
+  // dependent runs it before waiting for the kernel ahead of it, so that it
+  // overlaps that kernel's tail.
   template <class Policy>
-  __device__ __forceinline__ void init(unsigned char *smem_raw, uint32_t *status, Policy &pol,
-                                       int num_tiles) {
+  __device__ __forceinline__ void setup(unsigned char *smem_raw, const Policy &pol) {
     using namespace sm100;
     const uint32_t raw = smem_addr(smem_raw);
     base = (raw + 1023u) & ~1023u;
     smem = smem_raw + (base - raw);
     warp = threadIdx.x >> 5;
     lane = threadIdx.x & 31;
-    pol.prepare(smem);  // per-CTA tables of the policy (all threads)
-    if (warp >= 2) {    // half of this row's query into the swizzled Q tile (zeros past the end)
-      const int r = row_in_tile();
-      constexpr int kChunks = D / 16;  // 16-byte chunks per half row
-      const int c0 = group() * kChunks;
-      const uint4 *src = reinterpret_cast<const uint4 *>(pol.q_row(r));
-      uint4 v[kChunks];
-#pragma unroll
-      for (int i = 0; i < kChunks; ++i) v[i] = src ? __ldg(src + c0 + i) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int i = 0; i < kChunks; ++i) {
-        const int c = c0 + i;
-        *reinterpret_cast<uint4 *>(smem + L::kOffQ + (c >> 3) * L::kQHalf + sw128_offset(r, c & 7)) = v[i];
-      }
-      fence_proxy_async_smem();
-    }
     if (threadIdx.x == 0) {
       for (int st = 0; st < STAGES; ++st) {
         mbar_init(kv_full(st), 1);
@@ -150,13 +134,39 @@ struct Engine {
       mbar_init(user_bar(), 1);
       *abort_flag() = 0;
       fence_mbar_init();
-      // thread 0 is the producer: the first tiles' loads go out right away
-      if (Policy::kIssueBeforeSync && num_tiles > 0) issue_first(pol, num_tiles);
+      pol.prefetch();
     }
     if (warp == 1) {
       tmem_alloc(base + L::kOffMisc, L::kTmemCols);
       tmem_relinquish();
     }
+  }
+
+  // The data part of the set-up, after setup(): the policy's per-CTA tables, the
+  // query rows copied by the softmax threads into the Q tile, and (for a policy
+  // that allows it) the producer's loads of the first STAGES tiles, all before
+  // the CTA-wide barrier.
+  template <class Policy>
+  __device__ __forceinline__ void init(uint32_t *status, Policy &pol, int num_tiles) {
+    using namespace sm100;
+    pol.prepare(smem);  // per-CTA tables of the policy (all threads)
+    if (warp >= 2) {    // half of this row's query into the swizzled Q tile (zeros past the end)
+      const int r = row_in_tile();
+      constexpr int kChunks = D / 16;  // 16-byte chunks per half row
+      const int c0 = group() * kChunks;
+      const uint4 *src = reinterpret_cast<const uint4 *>(pol.q_row(r));
+      uint4 v[kChunks];
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) v[i] = src ? __ldg(src + c0 + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int c = c0 + i;
+        *reinterpret_cast<uint4 *>(smem + L::kOffQ + (c >> 3) * L::kQHalf + sw128_offset(r, c & 7)) = v[i];
+      }
+      fence_proxy_async_smem();
+    }
+    // thread 0 is the producer: the first tiles' loads go out right away
+    if (Policy::kIssueBeforeSync && threadIdx.x == 0 && num_tiles > 0) issue_first(pol, num_tiles);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -171,7 +181,6 @@ struct Engine {
 
   template <class Policy>
   __device__ __forceinline__ void issue_first(Policy &pol, int num_tiles) {
-    pol.prefetch();
     for (int k = 0; k < min(STAGES, num_tiles); ++k)
       pol.load_tile(k, stage_k(k), stage_v(k), L::kKVHalf, kv_full(k));
     DSA_TRACE_EVENT(2);
