@@ -72,38 +72,41 @@ struct SelectPolicy {
     sm100::tma_prefetch_map(kmap4);
     sm100::tma_prefetch_map(vmap4);
   }
+  // Run by all 32 lanes of warp 0: lanes 0..kPages-1 resolve one page each,
+  // lane 0 arms the barrier, then each box of the tile is issued by a lane of
+  // its own (one warp instruction for the tile).
   __device__ __forceinline__ void load_tile(int k, uint32_t sk, uint32_t sv, uint32_t half_bytes,
-                                            uint32_t bar) const {
+                                            uint32_t bar, int lane) const {
     constexpr int kPages = tc::kBN / PAGE;
+    constexpr int kHalves = D / 64;
     const int lp0 = (t_begin + k) * tc::kBN / PAGE;
-    long long phys[kPages];
-    uint32_t nvalid = 0;
-    bool run = true;  // all pages valid and physically consecutive
-#pragma unroll
-    for (int pi = 0; pi < kPages; ++pi) {
-      phys[pi] = phys_of(lp0 + pi);
-      if (phys[pi] >= 0) ++nvalid;
-      else if (lp0 + pi < np && blockIdx.x == 0) raise_status(status, kStatusBadIndex);
-      run = run && phys[pi] >= 0 && phys[pi] == phys[0] + pi;
-    }
-    sm100::mbar_arrive_expect_tx(bar, nvalid * PAGE * 128u * (D / 64) * 2u);
-    if (kPages > 1 && run) {  // the whole tile in one box per half
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        sm100::tma_load_4d(sk + hf * half_bytes, kmap4, bar, hf * 64, 0, h, (int)phys[0]);
-        sm100::tma_load_4d(sv + hf * half_bytes, vmap4, bar, hf * 64, 0, h, (int)phys[0]);
+    const long long my = phys_of(lp0 + (lane < kPages ? lane : 0));
+    const bool valid = lane < kPages && my >= 0;
+    if (lane < kPages && my < 0 && lp0 + lane < np && blockIdx.x == 0)
+      raise_status(status, kStatusBadIndex);
+    const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+    const long long p0 = __shfl_sync(0xffffffffu, my, 0);
+    const bool consec = lane >= kPages || (valid && my == p0 + lane);
+    const bool run = kPages > 1 && __all_sync(0xffffffffu, consec);
+    if (lane == 0)
+      sm100::mbar_arrive_expect_tx(bar, (uint32_t)__popc(vmask) * PAGE * 128u * kHalves * 2u);
+    if (run) {  // the whole tile in one box per half and tensor
+      if (lane < 2 * kHalves) {
+        const int hf = lane % kHalves;
+        const bool isv = lane >= kHalves;
+        sm100::tma_load_4d((isv ? sv : sk) + hf * half_bytes, isv ? vmap4 : kmap4, bar, hf * 64, 0, h,
+                           (int)p0);
       }
       return;
     }
-#pragma unroll
-    for (int pi = 0; pi < kPages; ++pi) {
-      if (phys[pi] < 0) continue;
-      const int y = (int)((phys[pi] * Hkv + h) * PAGE);
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        sm100::tma_load_2d(sk + hf * half_bytes + pi * PAGE * 128, kmap, bar, hf * 64, y);
-        sm100::tma_load_2d(sv + hf * half_bytes + pi * PAGE * 128, vmap, bar, hf * 64, y);
-      }
+    const int pi = lane / (2 * kHalves), rem = lane % (2 * kHalves);
+    const long long ph = __shfl_sync(0xffffffffu, my, pi < kPages ? pi : 0);
+    if (pi < kPages && ((vmask >> pi) & 1u)) {
+      const int hf = rem % kHalves;
+      const bool isv = rem >= kHalves;
+      const int y = (int)((ph * Hkv + h) * PAGE);
+      sm100::tma_load_2d((isv ? sv : sk) + hf * half_bytes + pi * PAGE * 128, isv ? vmap : kmap, bar,
+                         hf * 64, y);
     }
   }
   __device__ __forceinline__ const __nv_bfloat16 *q_row(int r) const {

@@ -50,8 +50,12 @@ struct MergeLayout {
   static __host__ __device__ constexpr uint32_t table_offset(int C) {
     return align16(weights_offset(C) + (uint32_t)(rpc(C) * C + 16) * 4u);
   }
+  // uint64 key mask per page tile, after the table
+  static __host__ __device__ constexpr uint32_t mask_offset(int C, int ppc) {
+    return table_offset(C) + 8u * (uint32_t)ppc;
+  }
   static __host__ __device__ constexpr size_t smem(int C, int ppc) {
-    return table_offset(C) + 8u * (uint32_t)ppc + 1024u;  // + alignment slack
+    return mask_offset(C, ppc) + 8u * (uint32_t)ppc + 1024u;  // + alignment slack
   }
 };
 
@@ -63,25 +67,27 @@ struct SparseParams {
 
 template <int D, int PAGE>
 struct SparsePolicy {
-  // the CTA's selected pages are resolved into a shared-memory table of
-  // (logical page, physical page) during set-up; until that table is complete
-  // (only the producer's first loads) entries are read directly
+  // warp 0 resolves the CTA's selected pages into a shared-memory table of
+  // (logical page, physical page) and a key mask per page tile during set-up,
+  // before it issues the first loads; the other warps read both after the
+  // CTA-wide barrier
   static constexpr bool kIssueBeforeSync = true;
   static constexpr int kPagesPerTile = tc::kBN / PAGE;
+  static constexpr int kHalves = D / 64;
   const CUtensorMap *kmap, *vmap, *kmap4, *vmap4, *bkmap, *bvmap;
   const int32_t *idx_row;       // idx[s, h, :]
   const int32_t *page_row;      // page-table row of the sequence, or null (identity)
   const __nv_bfloat16 *q_head;  // q[s, 0, h*G, 0]
   uint32_t *status;
   const int2 *tab;              // shared: (lp, phys) per entry of this CTA, phys < 0 = unusable
-  uint32_t tab_off;             // byte offset of the table in the aligned shared memory
-  bool table_ready;
+  const uint64_t *masks;        // shared: key mask of each page tile
+  uint32_t tab_off, mask_off;   // byte offsets in the aligned shared memory
+  int lp_spec;                  // warp 0: idx[s, h, c*ppc + lane], loaded with idx_cnt
   long long n_phys, phys0;
   int Hkv, h, G, Hq, B, BG, s, n, np, e_begin, e_end, sel_tiles, row_base;
   float sl2;
 
-  __device__ __forceinline__ int2 resolve(int e) const {
-    const int lp = idx_row[e];
+  __device__ __forceinline__ int2 resolve_lp(int lp) const {
     int phys = -1;
     if (lp >= 0 && lp < np) {
       const long long p = page_row ? (long long)page_row[lp] : phys0 + lp;
@@ -91,15 +97,36 @@ struct SparsePolicy {
   }
   __device__ __forceinline__ void prepare(unsigned char *smem) {
     int2 *t = reinterpret_cast<int2 *>(smem + tab_off);
-    for (int e = e_begin + (int)threadIdx.x; e < e_end; e += (int)blockDim.x) {
-      const int2 v = resolve(e);
-      if (v.y < 0) raise_status(status, kStatusBadIndex);
-      t[e - e_begin] = v;
-    }
+    uint64_t *mk = reinterpret_cast<uint64_t *>(smem + mask_off);
     tab = t;
-    table_ready = false;
+    masks = mk;
+    if (threadIdx.x >= 32) return;
+    const int lane = threadIdx.x;
+    // e_begin == c * ppc whenever the slice is not empty, so entry i = lane of the
+    // first pass is the one loaded speculatively
+    for (int i = lane; i < e_end - e_begin; i += 32) {
+      const int lp = i == lane ? lp_spec : idx_row[e_begin + i];
+      const int2 v = resolve_lp(lp);
+      if (v.y < 0) raise_status(status, kStatusBadIndex);
+      t[i] = v;
+    }
+    __syncwarp();
+    for (int k = lane; k < sel_tiles; k += 32) {
+      uint64_t m = 0;
+#pragma unroll
+      for (int pi = 0; pi < kPagesPerTile; ++pi) {
+        const int e = e_begin + k * kPagesPerTile + pi;
+        if (e >= e_end) continue;
+        const int2 v = t[e - e_begin];
+        if (v.y < 0) continue;
+        const int cnt = min(PAGE, n - v.x * PAGE);
+        if (cnt > 0) m |= ((cnt >= 64) ? ~0ull : ((1ull << cnt) - 1ull)) << (pi * PAGE);
+      }
+      mk[k] = m;
+    }
+    __syncwarp();
   }
-  __device__ __forceinline__ void ready() { table_ready = true; }
+  __device__ __forceinline__ void ready() const {}
   __device__ __forceinline__ void prefetch() const {
     sm100::tma_prefetch_map(kmap);
     sm100::tma_prefetch_map(vmap);
@@ -110,47 +137,48 @@ struct SparsePolicy {
   }
   __device__ __forceinline__ int2 entry(int e) const {
     if (e >= e_end) return make_int2(-1, -1);
-    return table_ready ? tab[e - e_begin] : resolve(e);
+    return tab[e - e_begin];
   }
+  // Run by all 32 lanes of warp 0: lane 0 arms the barrier, then each box of the
+  // tile is issued by a lane of its own (one warp instruction for the tile).
   __device__ __forceinline__ void load_tile(int k, uint32_t sk, uint32_t sv, uint32_t half_bytes,
-                                            uint32_t bar) const {
+                                            uint32_t bar, int lane) const {
     if (k < sel_tiles) {
       const int e0 = e_begin + k * kPagesPerTile;
-      int phys[kPagesPerTile];
-      uint32_t nvalid = 0;
-      bool run = true;  // all pages usable and physically consecutive
-#pragma unroll
-      for (int pi = 0; pi < kPagesPerTile; ++pi) {
-        phys[pi] = entry(e0 + pi).y;
-        nvalid += phys[pi] >= 0;
-        run = run && phys[pi] >= 0 && phys[pi] == phys[0] + pi;
-      }
-      sm100::mbar_arrive_expect_tx(bar, nvalid * PAGE * 128u * (D / 64) * 2u);
-      if (kPagesPerTile > 1 && run) {  // the whole tile in one box per half
-#pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf) {
-          sm100::tma_load_4d(sk + hf * half_bytes, kmap4, bar, hf * 64, 0, h, phys[0]);
-          sm100::tma_load_4d(sv + hf * half_bytes, vmap4, bar, hf * 64, 0, h, phys[0]);
+      const int2 my = entry(e0 + (lane < kPagesPerTile ? lane : 0));
+      const bool valid = lane < kPagesPerTile && my.y >= 0;
+      const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+      const int p0 = __shfl_sync(0xffffffffu, my.y, 0);
+      const bool consec = lane >= kPagesPerTile || (valid && my.y == p0 + lane);
+      const bool run = kPagesPerTile > 1 && __all_sync(0xffffffffu, consec);
+      if (lane == 0)
+        sm100::mbar_arrive_expect_tx(bar, (uint32_t)__popc(vmask) * PAGE * 128u * kHalves * 2u);
+      if (run) {  // the whole tile in one box per half and tensor
+        if (lane < 2 * kHalves) {
+          const int hf = lane % kHalves;
+          const bool isv = lane >= kHalves;
+          sm100::tma_load_4d((isv ? sv : sk) + hf * half_bytes, isv ? vmap4 : kmap4, bar, hf * 64, 0,
+                             h, p0);
         }
         return;
       }
-#pragma unroll
-      for (int pi = 0; pi < kPagesPerTile; ++pi) {
-        if (phys[pi] < 0) continue;
-        const int y = (int)(((long long)phys[pi] * Hkv + h) * PAGE);
-#pragma unroll
-        for (int hf = 0; hf < D / 64; ++hf) {
-          sm100::tma_load_2d(sk + hf * half_bytes + pi * PAGE * 128, kmap, bar, hf * 64, y);
-          sm100::tma_load_2d(sv + hf * half_bytes + pi * PAGE * 128, vmap, bar, hf * 64, y);
-        }
+      const int pi = lane / (2 * kHalves), rem = lane % (2 * kHalves);
+      const int ph = __shfl_sync(0xffffffffu, my.y, pi < kPagesPerTile ? pi : 0);
+      if (pi < kPagesPerTile && ((vmask >> pi) & 1u)) {
+        const int hf = rem % kHalves;
+        const bool isv = rem >= kHalves;
+        const int y = (int)(((long long)ph * Hkv + h) * PAGE);
+        sm100::tma_load_2d((isv ? sv : sk) + hf * half_bytes + pi * PAGE * 128, isv ? vmap : kmap, bar,
+                           hf * 64, y);
       }
     } else {  // the block's own tokens u = 64j .. 64j+63 of this sequence
       const int j = k - sel_tiles;
-      sm100::mbar_arrive_expect_tx(bar, 64u * 128u * (D / 64) * 2u);
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        sm100::tma_load_3d(sk + hf * half_bytes, bkmap, bar, hf * 64, h, s * B + j * 64);
-        sm100::tma_load_3d(sv + hf * half_bytes, bvmap, bar, hf * 64, h, s * B + j * 64);
+      if (lane == 0) sm100::mbar_arrive_expect_tx(bar, 64u * 128u * kHalves * 2u);
+      if (lane < 2 * kHalves) {
+        const int hf = lane % kHalves;
+        const bool isv = lane >= kHalves;
+        sm100::tma_load_3d((isv ? sv : sk) + hf * half_bytes, isv ? bvmap : bkmap, bar, hf * 64, h,
+                           s * B + j * 64);
       }
     }
   }
@@ -161,21 +189,9 @@ struct SparsePolicy {
     return q_head + ((size_t)b * Hq + g) * D;
   }
   __device__ __forceinline__ uint64_t key_mask(int k) const {
-    uint64_t m = 0;
-    if (k < sel_tiles) {
-      const int e0 = e_begin + k * kPagesPerTile;
-#pragma unroll
-      for (int pi = 0; pi < kPagesPerTile; ++pi) {
-        const int2 t = entry(e0 + pi);
-        if (t.y < 0) continue;
-        const int cnt = min(PAGE, n - t.x * PAGE);
-        if (cnt > 0) m |= ((cnt >= 64) ? ~0ull : ((1ull << cnt) - 1ull)) << (pi * PAGE);
-      }
-    } else {
-      const int cnt = min(64, B - (k - sel_tiles) * 64);
-      if (cnt > 0) m = (cnt >= 64) ? ~0ull : ((1ull << cnt) - 1ull);
-    }
-    return m;
+    if (k < sel_tiles) return masks[k];
+    const int cnt = min(64, B - (k - sel_tiles) * 64);
+    return cnt <= 0 ? 0ull : (cnt >= 64 ? ~0ull : ((1ull << cnt) - 1ull));
   }
   __device__ __forceinline__ void after_tile(int, int, float, const float *) const {}
 };
@@ -210,29 +226,44 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
   tc::Engine<D, kSpStages> eng;
   eng.setup(smem_raw, pol);
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(32);
   // everything below may read what the kernel ahead of this one wrote
   sm100::grid_dep_wait();
   sm100::grid_dep_launch_dependents();
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(33);
 
-  const bool reporter = threadIdx.x == 0 && c == 0 && rt == 0;
-  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status, reporter && h == 0);
+  // the prefix length, the count and (warp 0 of a page CTA) this CTA's slice of
+  // idx are loaded together: idx entries below kmax are always readable, and
+  // the ones beyond the count are ignored
+  const int32_t *idx_row = a.idx + sh_idx * sh.kmax;
+  const int n_raw = a.n_ctx[s];
   int cnt = a.idx_cnt[sh_idx];
+  int lp_spec = -1;
+  if (threadIdx.x < 32 && !blk_cta) {
+    const int e = c * plan.ppc + (int)threadIdx.x;
+    if ((int)threadIdx.x < plan.ppc && e < sh.kmax) lp_spec = idx_row[e];
+  }
+  const bool reporter = threadIdx.x == 0 && c == 0 && rt == 0;
+  const int n = clamp_prefix(n_raw, sh.max_pages, PAGE, a.status, reporter && h == 0);
   if (cnt < 0 || cnt > sh.kmax) {
     if (reporter) raise_status(a.status, kStatusBadIndex);
     cnt = max(0, min(cnt, sh.kmax));
   }
+  if (threadIdx.x == 0) DSA_TRACE_AFTER(34, cnt + n);
   const int e_begin = blk_cta ? cnt : min(cnt, c * plan.ppc);
   const int e_end = blk_cta ? cnt : min(cnt, (c + 1) * plan.ppc);
   const int sel_tiles = (e_end - e_begin + kPagesPerTile - 1) / kPagesPerTile;
   const int num_tiles = sel_tiles + (blk_cta ? plan.blk_tiles : 0);
 
-  pol.idx_row = a.idx + sh_idx * sh.kmax;
+  pol.idx_row = idx_row;
   pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
   pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
   pol.status = a.status;
   pol.tab = nullptr;
+  pol.masks = nullptr;
   pol.tab_off = M::table_offset(C);
-  pol.table_ready = false;
+  pol.mask_off = M::mask_offset(C, plan.ppc);
+  pol.lp_spec = lp_spec;
   pol.n_phys = sh.n_phys;
   pol.phys0 = (long long)s * sh.max_pages;
   pol.Hkv = sh.Hkv;

@@ -3,8 +3,10 @@
 // of 64-key tiles that a Policy describes.
 //
 // Warp roles (320 threads):
-//   warp 0      TMA producer: Policy::load_tile issues the tile's K and V boxes
-//               into a STAGES-deep ring of 128-byte-swizzled shared tiles;
+//   warp 0      TMA producer: Policy::load_tile, run by all 32 lanes, issues
+//               the tile's K and V boxes (one lane per box, so one warp
+//               instruction per tile) into a STAGES-deep ring of
+//               128-byte-swizzled shared tiles;
 //   warp 1      TMEM owner and MMA issuer: S_k = Q K_k^T into a double-buffered
 //               TMEM S (64 fp32 columns each), O += P_k V_k into TMEM O;
 //   warps 2..9  two softmax warpgroups that take alternate tiles (group g
@@ -150,6 +152,7 @@ struct Engine {
   __device__ __forceinline__ void init(uint32_t *status, Policy &pol, int num_tiles) {
     using namespace sm100;
     pol.prepare(smem);  // per-CTA tables of the policy (all threads)
+    if (threadIdx.x == 0) DSA_TRACE_EVENT(35);
     if (warp >= 2) {    // half of this row's query into the swizzled Q tile (zeros past the end)
       const int r = row_in_tile();
       constexpr int kChunks = D / 16;  // 16-byte chunks per half row
@@ -158,6 +161,7 @@ struct Engine {
       uint4 v[kChunks];
 #pragma unroll
       for (int i = 0; i < kChunks; ++i) v[i] = src ? __ldg(src + c0 + i) : make_uint4(0, 0, 0, 0);
+      if (r == 0 && group() == 0) DSA_TRACE_AFTER(37, v[0].x);
 #pragma unroll
       for (int i = 0; i < kChunks; ++i) {
         const int c = c0 + i;
@@ -166,24 +170,27 @@ struct Engine {
       fence_proxy_async_smem();
     }
     // thread 0 is the producer: the first tiles' loads go out right away
-    if (Policy::kIssueBeforeSync && threadIdx.x == 0 && num_tiles > 0) issue_first(pol, num_tiles);
+    if (Policy::kIssueBeforeSync && warp == 0 && num_tiles > 0) issue_first(pol, num_tiles);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     pol.ready();  // tables built by prepare() are complete from here on
     // (a policy whose first tile addresses need those tables issues them now)
-    if (!Policy::kIssueBeforeSync && threadIdx.x == 0 && num_tiles > 0) issue_first(pol, num_tiles);
+    if (!Policy::kIssueBeforeSync && warp == 0 && num_tiles > 0) issue_first(pol, num_tiles);
     tmem = *reinterpret_cast<volatile uint32_t *>(smem + L::kOffMisc);
     ctx = sm100::WaitCtx{abort_flag(), status};
     if (warp >= 2) mbar_arrive(q_full());
     if (threadIdx.x == 0) DSA_TRACE_EVENT(1);
   }
 
+  // Loads of the first STAGES tiles; all 32 lanes of warp 0 (the policy issues a
+  // tile's boxes from several lanes at once).
   template <class Policy>
   __device__ __forceinline__ void issue_first(Policy &pol, int num_tiles) {
+    if (lane == 0) DSA_TRACE_EVENT(36);
     for (int k = 0; k < min(STAGES, num_tiles); ++k)
-      pol.load_tile(k, stage_k(k), stage_v(k), L::kKVHalf, kv_full(k));
-    DSA_TRACE_EVENT(2);
+      pol.load_tile(k, stage_k(k), stage_v(k), L::kKVHalf, kv_full(k), lane);
+    if (lane == 0) DSA_TRACE_EVENT(2);
   }
 
   // Runs the pipeline over `num_tiles` tiles.  Softmax threads return their
@@ -200,18 +207,19 @@ struct Engine {
     l_out = 0.f;
     if (warp == 0) {
       // ---------------------------------------------------------- producer --
-      if (lane == 0 && num_tiles > 0) {
+      if (num_tiles > 0) {  // the whole warp: a tile's boxes go out from several lanes
         int issued = min(STAGES, num_tiles);  // issued during init
         for (int k = issued; k < num_tiles; ++k) {
           const int st = k % STAGES;
-          if (!mbar_wait(kv_empty(st), ((k / STAGES) - 1) & 1, ctx)) break;
-          pol.load_tile(k, stage_k(st), stage_v(st), L::kKVHalf, kv_full(st));
-          if (k == STAGES) DSA_TRACE_EVENT(24);
+          if (!__all_sync(0xffffffffu, mbar_wait(kv_empty(st), ((k / STAGES) - 1) & 1, ctx))) break;
+          pol.load_tile(k, stage_k(st), stage_v(st), L::kKVHalf, kv_full(st), lane);
+          if (k == STAGES && lane == 0) DSA_TRACE_EVENT(24);
           issued = k + 1;
         }
         // copies in flight land before the CTA's shared memory is released
-        for (int k = max(0, issued - STAGES); k < issued; ++k)
-          mbar_wait(kv_full(k % STAGES), (k / STAGES) & 1, drain_ctx);
+        if (lane == 0)
+          for (int k = max(0, issued - STAGES); k < issued; ++k)
+            mbar_wait(kv_full(k % STAGES), (k / STAGES) & 1, drain_ctx);
       }
     } else if (warp == 1) {
       // --------------------------------------------------------- MMA issuer --

@@ -11,7 +11,7 @@
 #include "sm100.cuh"
 
 namespace dsa {
-constexpr int kTraceEvents = 32;
+constexpr int kTraceEvents = 48;
 constexpr int kTraceCtas = 4096;
 }  // namespace dsa
 
@@ -22,6 +22,12 @@ static __device__ unsigned long long g_dsa_trace[dsa::kTraceCtas * dsa::kTraceEv
     const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
     if (cta_ < (unsigned)::dsa::kTraceCtas)                                                \
       g_dsa_trace[cta_ * ::dsa::kTraceEvents + (ev)] = ::dsa::sm100::global_ns();          \
+  } while (0)
+// stamp once `val` (a loaded value) is available: the empty asm consumes it
+#define DSA_TRACE_AFTER(ev, val)                         \
+  do {                                                   \
+    asm volatile("" ::"r"((unsigned)(val)) : "memory");  \
+    DSA_TRACE_EVENT(ev);                                 \
   } while (0)
 #define DSA_TRACE_EXPORT(fn)                                                         \
   extern "C" int fn(void *host, size_t bytes) {                                     \
@@ -36,6 +42,9 @@ static __device__ unsigned long long g_dsa_trace[dsa::kTraceCtas * dsa::kTraceEv
 #else
 #define DSA_TRACE_EVENT(ev) \
   do {                      \
+  } while (0)
+#define DSA_TRACE_AFTER(ev, val) \
+  do {                           \
   } while (0)
 #define DSA_TRACE_EXPORT(fn)
 #endif
