@@ -254,6 +254,7 @@ int dsa_sparse_attn(const void *q_blk, const void *k_cache, const void *v_cache,
   a.n_ctx = n_ctx;
   a.o_out = static_cast<__nv_bfloat16 *>(o_out);
   a.status = at<uint32_t>(workspace, 0);
+  a.xchg = at<unsigned char>(workspace, plan.off_xchg);
   if (dsa::launch_sparse(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;

@@ -69,7 +69,9 @@ struct SparsePlan {
   int cluster;    // CTAs per (seq, KV head, row tile): one thread-block cluster
   int ppc;        // selected pages per CTA of the cluster
   int blk_tiles;  // ceil(B / 64): tiles over the block's own tokens (last CTA)
-  size_t total;   // workspace bytes (status word)
+  size_t off_xchg;    // workspace offset of the partial-row exchange area
+  size_t xchg_slot;   // bytes of one CTA's partial rows in that area
+  size_t total;       // workspace bytes
 };
 
 struct SparseArgs {
@@ -77,6 +79,7 @@ struct SparseArgs {
   const int32_t *idx, *idx_cnt, *n_ctx;
   __nv_bfloat16 *o_out;
   uint32_t *status;
+  unsigned char *xchg;  // partial rows of every cluster, [S][Hkv][rowtiles][16 slots]
 };
 
 SparsePlan plan_sparse(const Shape &sh, int num_sms);

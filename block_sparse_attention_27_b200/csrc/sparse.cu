@@ -9,10 +9,12 @@
 // their slices [c*ppc, (c+1)*ppc) of the selected pages, gathered with TMA
 // through the page table; CTA C-1 takes the block's own tokens (a 3-D TMA box
 // over blk_k / blk_v), so that no CTA carries both.  The C partial results are
-// then merged inside the cluster: every CTA pushes each owner CTA the rows that
-// owner writes (its normalised output rows in fp16 plus the row max and sum),
-// with bulk copies into the owner's receive buffer, and each owner combines the
-// C contributions of its rows and writes them to o_out in bf16.
+// then merged: every softmax thread writes its row, normalised, in fp16 with
+// the row's (m, l), to this cluster's exchange area in the workspace (L2); after
+// one cluster barrier (release / acquire) the CTA that owns a row reads the C
+// contributions of its rows, combines them and writes o_out in bf16.  The
+// cluster only provides the co-scheduling and the barrier: going through L2
+// moves the partial rows faster than stores into the owners' shared memory.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -28,34 +30,23 @@ constexpr int kSpStages = 2;
 constexpr int kRowsPerCta = 128;
 constexpr int kMaxCluster = 16;
 
-// Exchange buffers of the cluster merge.  A row is a CTA's normalised output row
-// O/l in fp16 (D values) followed by (m, l, -, -) in fp32.  CTA j owns rows
-// [j*rpc, min(128, (j+1)*rpc)) with rpc = ceil(128 / C); its receive buffer has
-// one slot of rpc rows per source CTA and lies after every region the attention
-// engine uses, so data from a CTA that finished early cannot land on tiles that
-// are still being read.  The merge weights (one per owned row and source) and
-// the CTA's page table follow it.
+// Shared memory beyond the engine's layout: the CTA's page table (int2 per
+// entry) and a uint64 key mask per page tile.  Exchange area of one cluster in
+// the workspace: kMaxCluster slots (one per CTA), each the CTA's 128 partial rows
+// as [D/8 column chunks][128 rows][16 bytes] of fp16 (so a warp's stores of one
+// chunk are contiguous) followed by [128 rows] of (m, l) in fp32.
 template <int D>
-struct MergeLayout {
-  static constexpr uint32_t kRowBytes = D * 2 + 16;
-  static __host__ __device__ constexpr uint32_t recv_offset() {
-    return (tc::Layout<D, kSpStages>::kBytes + 1023u) & ~1023u;
-  }
-  static __host__ __device__ constexpr uint32_t rpc(int C) { return (kRowsPerCta + C - 1) / C; }
+struct SparseLayout {
+  static constexpr uint32_t kSlotBytes = 128u * (2u * D + 8u);
   static __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
-  static __host__ __device__ constexpr uint32_t weights_offset(int C) {
-    return align16(recv_offset() + (uint32_t)C * rpc(C) * kRowBytes);
+  static __host__ __device__ constexpr uint32_t table_offset() {
+    return align16(tc::Layout<D, kSpStages>::kBytes);
   }
-  // int2 entries: the offset must stay 8-byte (here 16-byte) aligned whatever C is
-  static __host__ __device__ constexpr uint32_t table_offset(int C) {
-    return align16(weights_offset(C) + (uint32_t)(rpc(C) * C + 16) * 4u);
+  static __host__ __device__ constexpr uint32_t mask_offset(int ppc) {
+    return table_offset() + 8u * (uint32_t)ppc;
   }
-  // uint64 key mask per page tile, after the table
-  static __host__ __device__ constexpr uint32_t mask_offset(int C, int ppc) {
-    return table_offset(C) + 8u * (uint32_t)ppc;
-  }
-  static __host__ __device__ constexpr size_t smem(int C, int ppc) {
-    return mask_offset(C, ppc) + 8u * (uint32_t)ppc + 1024u;  // + alignment slack
+  static __host__ __device__ constexpr size_t smem(int ppc) {
+    return mask_offset(ppc) + 8u * (uint32_t)ppc + 1024u;  // + alignment slack
   }
 };
 
@@ -202,7 +193,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kmap4,
                 const __grid_constant__ CUtensorMap vmap4, const __grid_constant__ CUtensorMap bkmap,
                 const __grid_constant__ CUtensorMap bvmap) {
-  using M = MergeLayout<D>;
+  using M = SparseLayout<D>;
   extern __shared__ unsigned char smem_raw[];
   const Shape &sh = prm.sh;
   const SparsePlan &plan = prm.plan;
@@ -261,8 +252,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.status = a.status;
   pol.tab = nullptr;
   pol.masks = nullptr;
-  pol.tab_off = M::table_offset(C);
-  pol.mask_off = M::mask_offset(C, plan.ppc);
+  pol.tab_off = M::table_offset();
+  pol.mask_off = M::mask_offset(plan.ppc);
   pol.lp_spec = lp_spec;
   pol.n_phys = sh.n_phys;
   pol.phys0 = (long long)s * sh.max_pages;
@@ -281,33 +272,30 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.row_base = row_base;
   pol.sl2 = sh.sl2;
   eng.init(a.status, pol, num_tiles);
-  // rows this CTA owns in the merge, and the bytes it will receive for them
-  const int rpc = (int)M::rpc(C);
+  // rows this CTA owns in the merge
+  const int rpc = (kRowsPerCta + C - 1) / C;
   const int r0 = c * rpc;
   const int nrows = max(0, min(kRowsPerCta, r0 + rpc) - r0);
-  if (threadIdx.x == 0)
-    sm100::mbar_arrive_expect_tx(eng.user_bar(), (uint32_t)(C * nrows) * M::kRowBytes);
-  sm100::cluster_arrive();  // barrier init and expected bytes are visible to the cluster
 
   float m, l;
   eng.template run<PAGE>(pol, num_tiles, m, l);
   float m_row, l_row, wa, wb;
   eng.finish(m, l, m_row, l_row, wa, wb);
 
-  // ---- stage: this CTA's rows, normalised (O / l) in fp16, with (m, l) in fp32,
-  //      into the send buffer (the Q / K/V area, free now that every MMA is done)
-  unsigned char *sendb = eng.smem;
+  // ---- exchange: each softmax thread writes its half of its row, normalised
+  //      (O / l) in fp16, to this CTA's slot of the cluster's exchange area; the
+  //      group-0 thread adds the row's (m, l)
+  unsigned char *xc = a.xchg + (((size_t)s * sh.Hkv + h) * plan.rowtiles + rt) * kMaxCluster * M::kSlotBytes;
   if (eng.warp >= 2) {
     const int r = eng.row_in_tile();
     const int g = eng.group();
+    unsigned char *slot = xc + (size_t)c * M::kSlotBytes;
     const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
     const float ca = wa * inv, cb = wb * inv;
-    unsigned char *row = sendb + r * M::kRowBytes;
 #pragma unroll
     for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 32) {
       uint32_t oa[32], ob[32];
-      eng.load_o(0, c0, oa);
-      eng.load_o(1, c0, ob);
+      eng.load_o2(c0, oa, ob);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint4 v;
@@ -318,92 +306,83 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 #pragma unroll
           for (int z = 0; z < 2; ++z) {
             const int i = 8 * q + 2 * e + z;
+            // an empty group (weight 0) may hold stale TMEM: never multiply it
             f[z] = (ca > 0.f ? ca * __uint_as_float(oa[i]) : 0.f) +
                    (cb > 0.f ? cb * __uint_as_float(ob[i]) : 0.f);
           }
           __half2 hv = __floats2half2_rn(f[0], f[1]);
           pv[e] = *reinterpret_cast<uint32_t *>(&hv);
         }
-        *reinterpret_cast<uint4 *>(row + c0 * 2 + q * 16) = v;
+        const int ch = c0 / 8 + q;
+        *reinterpret_cast<uint4 *>(slot + ((size_t)ch * kRowsPerCta + r) * 16) = v;
       }
     }
-    if (g == 0) *reinterpret_cast<float4 *>(row + D * 2) = make_float4(m_row, l_row, 0.f, 0.f);
-    sm100::fence_proxy_async_smem();
+    if (g == 0)
+      *reinterpret_cast<float2 *>(slot + (size_t)kRowsPerCta * 2 * D + r * 8) = make_float2(m_row, l_row);
     if (r == 0 && g == 0) DSA_TRACE_EVENT(7);
   }
-  __syncthreads();
-  sm100::cluster_wait();  // every CTA of the cluster has armed its receive barrier
-  if (threadIdx.x == 0) DSA_TRACE_EVENT(8);
-  const uint32_t recv = eng.base + M::recv_offset();
-  if (threadIdx.x == 0) {
-    const uint32_t send = smem_addr(sendb);
-    for (int j = 0; j < C; ++j) {
-      const int jr0 = j * rpc;
-      const int jn = max(0, min(kRowsPerCta, jr0 + rpc) - jr0);
-      if (jn == 0) continue;
-      sm100::bulk_copy_to_cluster(sm100::cluster_map(recv + c * rpc * M::kRowBytes, j),
-                                  send + jr0 * M::kRowBytes, jn * M::kRowBytes,
-                                  sm100::cluster_map(eng.user_bar(), j));
-    }
-    sm100::bulk_commit();
-  }
-
-  // ---- receive this CTA's rows from every CTA and merge them
-  const bool got = __syncthreads_and(sm100::mbar_wait(eng.user_bar(), 0, eng.ctx));
+  sm100::cluster_arrive();  // release: this CTA's partial rows are written
+  sm100::cluster_wait();    // acquire: so are those of every CTA of the cluster
   if (threadIdx.x == 0) DSA_TRACE_EVENT(9);
+
+  // ---- merge the rows this CTA owns: a work item (row, 8 columns) loads the C
+  //      contributions' (m, l) and values at once (L2 only: they come from other
+  //      SMs), then weighs them with 2^(m_j - M) l_j / L.  Consecutive threads
+  //      take consecutive rows of one column chunk, so that their loads are
+  //      contiguous in the chunk-major slots.
   const int rows_here = min(kRowsPerCta, sh.BG - row_base);
-  const unsigned char *rb = eng.smem + M::recv_offset();
-  float *wts = reinterpret_cast<float *>(eng.smem + M::weights_offset(C));  // [nrows][C]
-  for (int rl = threadIdx.x; got && rl < nrows; rl += blockDim.x) {
-    float mx = -INFINITY;
-    for (int j = 0; j < C; ++j) {
-      const float2 st = *reinterpret_cast<const float2 *>(rb + (j * rpc + rl) * M::kRowBytes + D * 2);
-      if (st.y > 0.f) mx = fmaxf(mx, st.x);
-    }
-    float lsum = 0.f;
-    for (int j = 0; j < C; ++j) {
-      const float2 st = *reinterpret_cast<const float2 *>(rb + (j * rpc + rl) * M::kRowBytes + D * 2);
-      const float w = st.y > 0.f ? exp2f(st.x - mx) * st.y : 0.f;  // 0: an empty partial
-      wts[rl * C + j] = w;
-      lsum += w;
-    }
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    for (int j = 0; j < C; ++j) wts[rl * C + j] *= inv;
-  }
-  __syncthreads();
   constexpr int kChunks = D / 8;  // 8 values (16 bytes of fp16) per work item
-  for (int t = threadIdx.x; got && t < nrows * kChunks; t += blockDim.x) {
-    const int rl = t / kChunks, ch = t % kChunks;
-    if (r0 + rl >= rows_here) continue;
+  for (int t = threadIdx.x; t < nrows * kChunks; t += blockDim.x) {
+    const int rl = t % nrows, ch = t / nrows;
+    const int row = r0 + rl;
+    if (row >= rows_here) continue;
+    float2 st[kMaxCluster];
+    uint4 v[kMaxCluster];
+#pragma unroll
+    for (int j = 0; j < kMaxCluster; ++j) {
+      if (j < C) {
+        const unsigned char *slot = xc + (size_t)j * M::kSlotBytes;
+        st[j] = __ldcg(reinterpret_cast<const float2 *>(slot + (size_t)kRowsPerCta * 2 * D + row * 8));
+        const int4 x = __ldcg(reinterpret_cast<const int4 *>(slot + ((size_t)ch * kRowsPerCta + row) * 16));
+        v[j] = make_uint4((uint32_t)x.x, (uint32_t)x.y, (uint32_t)x.z, (uint32_t)x.w);
+      } else {
+        st[j] = make_float2(-INFINITY, 0.f);
+        v[j] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kMaxCluster; ++j)
+      if (st[j].y > 0.f) mx = fmaxf(mx, st[j].x);
+    float lsum = 0.f;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < C; ++j) {
-      const float w = wts[rl * C + j];
-      if (w == 0.f) continue;
-      const uint4 v = *reinterpret_cast<const uint4 *>(rb + (j * rpc + rl) * M::kRowBytes + ch * 16);
-      const __half2 *hv = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+    for (int j = 0; j < kMaxCluster; ++j) {
+      if (!(st[j].y > 0.f)) continue;  // an empty contribution
+      const float w = exp2f(st[j].x - mx) * st[j].y;
+      lsum += w;
+      const __half2 *hv = reinterpret_cast<const __half2 *>(&v[j]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float2 f = __half22float2(hv[e]);
-        acc[2 * e] += w * f.x;
-        acc[2 * e + 1] += w * f.y;
+        acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
       }
     }
-    const int grow = row_base + r0 + rl;
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const int grow = row_base + row;
     const int b = grow / sh.G, g = grow % sh.G;
     uint4 outv;
     uint32_t *po = reinterpret_cast<uint32_t *>(&outv);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      __nv_bfloat162 bv = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+      __nv_bfloat162 bv = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
       po[e] = *reinterpret_cast<uint32_t *>(&bv);
     }
     *reinterpret_cast<uint4 *>(a.o_out + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D +
                                ch * 8) = outv;
   }
-  if (threadIdx.x == 0) {
-    DSA_TRACE_EVENT(10);
-    sm100::bulk_wait_read_all();  // outgoing copies have read the send buffer
-  }
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(10);
   eng.teardown();
   if (threadIdx.x == 0) DSA_TRACE_EVENT(11);
 }
@@ -468,17 +447,17 @@ inline int choose_page_ctas(const int *active, int nclusters, int kmax, int page
 template <int D, int PAGE>
 cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan_in, const SparseArgs &a,
                          cudaStream_t stream) {
-  using M = MergeLayout<D>;
+  using M = SparseLayout<D>;
   constexpr auto kern = sparse_attn<D, PAGE>;
   constexpr size_t kMaxSmem = 227 * 1024;
   cudaError_t err = set_smem_once<kern>(kMaxSmem);
   if (err != cudaSuccess) return err;
   SparsePlan plan = plan_in;
-  const int *active = active_clusters<kern>(M::smem(kMaxCluster, std::max(sh.kmax, 64)));
+  const int *active = active_clusters<kern>(M::smem(std::max(sh.kmax, 64)));
   const int cp = choose_page_ctas(active, sh.Hkv * sh.S * plan.rowtiles, sh.kmax, PAGE, plan.blk_tiles);
   plan.cluster = cp + 1;
   plan.ppc = (sh.kmax + cp - 1) / cp;
-  const size_t smem = M::smem(plan.cluster, plan.ppc);
+  const size_t smem = M::smem(plan.ppc);
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
   CUtensorMap kmap, vmap, kmap4, vmap4, bkmap, bvmap;
   const long long rows = sh.n_phys * sh.Hkv * PAGE;
@@ -525,7 +504,9 @@ SparsePlan plan_sparse(const Shape &sh, int /*num_sms*/) {
   p.cluster = kMaxCluster;  // refined at launch from the device's cluster capacity
   p.ppc = (sh.kmax + kMaxCluster - 2) / (kMaxCluster - 1);
   p.blk_tiles = (sh.B + tc::kBN - 1) / tc::kBN;
-  p.total = 4096;  // status word only: partials never leave the cluster
+  p.off_xchg = 4096;  // after the status header
+  p.xchg_slot = 128u * (2u * (size_t)sh.d + 8u);
+  p.total = p.off_xchg + (size_t)sh.S * sh.Hkv * p.rowtiles * kMaxCluster * p.xchg_slot;
   return p;
 }
 

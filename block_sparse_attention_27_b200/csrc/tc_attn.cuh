@@ -435,6 +435,10 @@ struct Engine {
   __device__ __forceinline__ void load_o(int which, int c0, uint32_t (&o)[32]) const {
     sm100::tmem_ld32(lane_tmem() + L::kTmemO + which * D + c0, o);
   }
+  // Columns [c0, c0+32) of both groups' O accumulators, with one wait.
+  __device__ __forceinline__ void load_o2(int c0, uint32_t (&o0)[32], uint32_t (&o1)[32]) const {
+    sm100::tmem_ld32x2(lane_tmem() + L::kTmemO + c0, o0, lane_tmem() + L::kTmemO + D + c0, o1);
+  }
 
   // All threads: waits for everybody, then the TMEM owner frees TMEM.
   __device__ __forceinline__ void teardown() {
