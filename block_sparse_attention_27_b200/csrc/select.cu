@@ -41,7 +41,7 @@ struct PartialParams {
 // and that max (mtile); the split's unnormalised O row, m and l go to part_o /
 // part_ml.
 // ---------------------------------------------------------------------------
-constexpr int kSelStages = 5;
+constexpr int kSelStages = 6;
 
 template <int D, int PAGE>
 struct SelectPolicy {

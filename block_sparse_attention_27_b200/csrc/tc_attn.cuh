@@ -15,7 +15,8 @@
 //               row r (TMEM lane r): online softmax in the log2 domain with lazy
 //               rescaling (the reference max moves only when a tile beats it by
 //               more than 2^8), per-unit sums (32 keys at most) handed to
-//               Policy::after_tile, P in bf16 to shared memory for the PV MMA.
+//               Policy::after_tile, P in bf16 into TMEM over the tile's S
+//               (the A operand of the PV MMA).
 //               Each group accumulates into its own TMEM O.
 // After run() every softmax thread holds its group's (m, l); finish() joins the
 // two groups' statistics, and the kernel combines the two O accumulators
@@ -54,18 +55,18 @@ struct Layout {
   static constexpr uint32_t kKVHalf = kBN * 128;          // 64 keys x 128 B
   static constexpr uint32_t kKBytes = kHalves * kKVHalf;
   static constexpr uint32_t kStageBytes = 2 * kKBytes;    // K tile then V tile
-  static constexpr uint32_t kPBytes = 128 * 128;          // 128 rows x 64 keys bf16
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = kOffQ + kHalves * kQHalf;
-  static constexpr uint32_t kOffP = kOffKV + STAGES * kStageBytes;
-  static constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
+  static constexpr uint32_t kOffBar = kOffKV + STAGES * kStageBytes;
   static constexpr int kNumBars = 2 * STAGES + 15;  // the last one is the kernel's own
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kOffML = kOffQ;  // [2 groups][128] (m, l), once Q is dead
   static constexpr uint32_t kBytes = kOffMisc + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;  // room to align the base to 1 KB
-  // TMEM: four S buffers of 64 columns (two per softmax group: buffer 2g+i),
-  // then the O accumulators of group 0 and group 1
+  // TMEM: four S buffers of 64 columns (two per softmax group: buffer 2g+i;
+  // the softmax overwrites the first 32 columns of a tile's buffer with its P
+  // in bf16, the A operand of the PV MMA), then the O accumulators of group 0
+  // and group 1
   static constexpr uint32_t kTmemO = 4 * kBN;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(D == 64 || D == 128, "head dimension");
@@ -259,11 +260,11 @@ struct Engine {
           if (j == 2) DSA_TRACE_EVENT(14);
           tc_fence_after();
           const uint32_t sv = stage_v(st);
+          const uint32_t pa = tmem + s_buf(j) * kBN;  // P_j in TMEM: 8 columns per 16 keys
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(base + L::kOffP + g * L::kPBytes + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(sv + kk * 16 * 128, L::kKVHalf, 1024);
-            umma_bf16(tmem + L::kTmemO + g * D, ad, bd, kIdO, (j > 1 || kk > 0) ? 1u : 0u);
+            umma_bf16_ts(tmem + L::kTmemO + g * D, pa + kk * 8, bd, kIdO, (j > 1 || kk > 0) ? 1u : 0u);
           }
           umma_commit(pv_done(g));
           umma_commit(kv_empty(st));
@@ -316,9 +317,9 @@ struct Engine {
         // tile max in the log2 domain (the scale is positive, so it commutes with max)
         const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * pol.sl2;
         if (tr) DSA_TRACE_EVENT(19);
-        // PV of this group's previous tile must have landed before O is rescaled
-        // or the group's P buffer is rewritten
-        bool pv_ready = mine == 0;
+        // PV of this group's previous tile must have landed before O is rescaled.
+        // (P goes into this tile's own S buffer, whose last reader, PV of the tile
+        // four earlier, was issued before this tile's S and hence is done.)
         const bool need = tmax > m_used + kRescaleLog2 || (m_used == -INFINITY && tmax > -INFINITY);
         if (__any_sync(0xffffffffu, need)) {
           float alpha = 1.f;
@@ -330,7 +331,6 @@ struct Engine {
           if (mine > 0) {  // O holds this group's earlier tiles: scale it
             alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 1) & 1, ctx));
             if (!alive) break;
-            pv_ready = true;
             tc_fence_after();
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
@@ -355,19 +355,11 @@ struct Engine {
 #pragma unroll
         for (int u = 0; u < U::kPerTile; ++u) l += usum[u];
         if (tr) DSA_TRACE_EVENT(20);
-        if (!pv_ready) {
-          alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 1) & 1, ctx));
-          if (!alive) break;
-        }
-        unsigned char *prow = smem + L::kOffP + g * L::kPBytes;
+        {  // P in bf16 over the first 32 columns of the tile's S buffer
+          uint32_t pk[kBN / 2];
 #pragma unroll
-        for (int c = 0; c < kBN / 8; ++c) {
-          uint4 v;
-          v.x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
-          v.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
-          v.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
-          v.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
-          *reinterpret_cast<uint4 *>(prow + sw128_offset(r, c)) = v;
+          for (int c = 0; c < kBN / 2; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
+          tmem_st32(lt + sb * kBN, pk);
         }
         if (tr) DSA_TRACE_EVENT(21);
         // value rows of keys that take no part are zeroed so that 0 * stale data
