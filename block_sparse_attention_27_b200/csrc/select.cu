@@ -3,13 +3,15 @@
 // KV head ("MAGE: All-[MASK] Block Already Knows Where to Look in Block
 // Diffusion LLM", Approach).
 //
-// Three launches on the caller's stream:
-//   1. select_partial: split-KV attention.  CTA = (split, row tile) x KV head x
-//      sequence; 8 warps x 16 rows = 128 query rows (b, g) of one KV head against
-//      the split's 64-token tiles, double-buffered with cp.async.  Per split it
+// Three launches on the caller's stream, each a programmatic dependent of the
+// one before it:
+//   1. select_partial: split-KV attention on the tcgen05 engine (tc_attn.cuh).
+//      CTA = (split, 128-row tile) x KV head x sequence, one wave over the SMs;
+//      the split's 64-token tiles stream through a TMA ring.  Per split it
 //      writes the unnormalised output O_j with its row max m_j and sum l_j, and
-//      per (page, row) the partial probability mass of the page relative to the
-//      running max at that tile (pagepart), together with that max (mtile).
+//      per (tile, row) the partial probability mass of each unit of the tile
+//      (min(page, 32) keys of one page) relative to the row's reference max at
+//      that tile (pagepart, [tile][row][unit]), together with that max (mtile).
 //   2. select_finalize: merges the splits into o_out and turns the partial
 //      masses into page scores  S_h[q] = (1/BG) sum_rows pagepart * 2^(mtile-M) / L.
 //   3. select_topk: radix select of the kp-th largest score per (seq, KV head),
@@ -41,7 +43,7 @@ struct PartialParams {
 // and that max (mtile); the split's unnormalised O row, m and l go to part_o /
 // part_ml.
 // ---------------------------------------------------------------------------
-constexpr int kSelStages = 6;
+constexpr int kSelStages = 5;
 
 template <int D, int PAGE>
 struct SelectPolicy {
@@ -53,7 +55,7 @@ struct SelectPolicy {
   const int32_t *page_row;          // page-table row of the sequence, or null (identity)
   const __nv_bfloat16 *q_head;      // q[s, 0, h*G, 0]
   float *mtile_head;                // mtile[s, h, 0, 0]
-  float *pagepart_head;             // pagepart[s, h, 0, 0]
+  float *pagepart_head;             // pagepart[s, h, 0, 0, 0]
   uint32_t *status;
   long long n_phys, phys0;          // phys0 = s*max_pages (identity map)
   int Hkv, h, G, Hq, BG, n, np, t_begin, row_base;
@@ -137,13 +139,12 @@ struct SelectPolicy {
     if (row >= BG) return;
     const int tile = t_begin + k;
     mtile_head[(size_t)tile * BG + row] = m_used;
-#pragma unroll
-    for (int u = 0; u < U::kPerTile; ++u) {
-      const int t = tile * tc::kBN + u * U::kKeys;
-      const int lp = t / PAGE;
-      if (lp < np)
-        pagepart_head[((size_t)lp * U::kPerPage + (t % PAGE) / U::kKeys) * BG + row] = usum[u];
-    }
+    // the row's unit masses of the tile, one vector store (units past the prefix hold 0)
+    float *dst = pagepart_head + ((size_t)tile * BG + row) * U::kPerTile;
+    if constexpr (U::kPerTile == 4)
+      *reinterpret_cast<float4 *>(dst) = make_float4(usum[0], usum[1], usum[2], usum[3]);
+    else
+      *reinterpret_cast<float2 *>(dst) = make_float2(usum[0], usum[1]);
   }
 };
 
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
   pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
   pol.mtile_head = a.mtile + sh_idx * plan.max_tiles * sh.BG;
-  pol.pagepart_head = a.pagepart + sh_idx * sh.max_pages * tc::Units<PAGE>::kPerPage * sh.BG;
+  pol.pagepart_head = a.pagepart + sh_idx * plan.max_tiles * sh.BG * tc::Units<PAGE>::kPerTile;
   pol.status = a.status;
   pol.n_phys = sh.n_phys;
   pol.phys0 = (long long)s * sh.max_pages;
@@ -242,7 +243,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // ---------------------------------------------------------------------------
 constexpr int kFinThreads = 256;
 constexpr int kRowsPerFinCta = 8;   // output CTAs: one query row per warp
-constexpr int kFinTiles = 2;        // score CTAs: 64-token tiles a warp loads at once
 constexpr int kFinBatch = 16;       // output CTAs: split partials a lane loads at once
 
 // Folds a partial (m, l) into the running (M, L) of a row (log2 domain); an
@@ -296,18 +296,47 @@ __device__ __forceinline__ void merged_row_stats(const Shape &sh, const SelectPl
   }
 }
 
+// Sum over the 32 lanes of a warp of the kP values v[0..kP) (kP = 1, 2 or 4)
+// with log2(32) + kP - 1 shuffles: the first rounds halve the set of values a
+// lane carries.  Value p ends in lane p * (32 / kP).
+template <int kP>
+__device__ __forceinline__ float warp_sum_multi(const float (&v)[kP], int lane) {
+  if constexpr (kP == 4) {
+    const bool hi = lane & 16;
+    const float s0 = hi ? v[0] : v[2], s1 = hi ? v[1] : v[3];
+    const float b0 = (hi ? v[2] : v[0]) + __shfl_xor_sync(0xffffffffu, s0, 16);
+    const float b1 = (hi ? v[3] : v[1]) + __shfl_xor_sync(0xffffffffu, s1, 16);
+    const bool h8 = lane & 8;
+    float c = (h8 ? b1 : b0) + __shfl_xor_sync(0xffffffffu, h8 ? b0 : b1, 8);
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    return c;
+  } else if constexpr (kP == 2) {
+    const bool hi = lane & 16;
+    float c = (hi ? v[1] : v[0]) + __shfl_xor_sync(0xffffffffu, hi ? v[0] : v[1], 16);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    return c;
+  } else {
+    return warp_sum(v[0]);
+  }
+}
+
 // Page scores of the pages [p0, p1) (tile-aligned) of one (sequence, KV head).
-// Lane i of a warp handles the rows VEC*i + 32*VEC*c (c < kChunks): their M and
-// 1/L stay in registers, and for kFinTiles tiles at a time the tile maxima and
-// every unit's partial masses are loaded before any of them is used.
-template <int PAGE, int VEC, int kChunks>
+// Lane i of a warp handles the rows VEC*i + 32*VEC*c + e (c < kChunks, e < VEC):
+// their M and 1/L stay in registers, and for kFinTiles tiles at a time the
+// tile maxima and each row's vector of unit masses are loaded before any of
+// them is used.
+template <int PAGE, int VEC, int kChunks, int kFinTiles>
 __device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &plan,
                                             const SelectArgs &a, size_t sh_idx, int np, int p0,
                                             int p1, const float *sM, const float *sLinv) {
   using U = tc::Units<PAGE>;
   using V = typename std::conditional<VEC == 4, float4, float>::type;
   constexpr int kPagesPerTile = tc::kBN / PAGE;
-  constexpr int kUnitsPerTile = U::kPerTile;
+  constexpr int kUnits = U::kPerTile;  // 4 or 2
+  using W = typename std::conditional<kUnits == 4, float4, float2>::type;
+  static_assert(kUnits == 4 || kUnits == 2, "units per tile");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int BG = sh.BG;
   float rm[kChunks][VEC], rl[kChunks][VEC];
@@ -319,42 +348,35 @@ __device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &p
       rm[c][e] = row < BG ? sM[row] : 0.f;
       rl[c][e] = row < BG ? sLinv[row] : 0.f;  // 0: the row does not exist
     }
-  auto load = [&](const float *base, int c) -> V {
-    const int row = VEC * lane + 32 * VEC * c;
-    if (row >= BG) {
-      V z;
-      memset(&z, 0, sizeof z);
-      return z;
-    }
-    return *reinterpret_cast<const V *>(base + row);
-  };
   auto lanes = [](const V &v, int e) -> float { return reinterpret_cast<const float *>(&v)[e]; };
+  auto units = [](const W &w, int u) -> float { return reinterpret_cast<const float *>(&w)[u]; };
   const float inv_bg = 1.f / (float)BG;
   const int warps = (int)blockDim.x / 32;
   const float *mt_head = a.mtile + sh_idx * plan.max_tiles * BG;
-  const float *pp_head = a.pagepart + sh_idx * sh.max_pages * U::kPerPage * BG;
+  const float *pp_head = a.pagepart + sh_idx * plan.max_tiles * BG * kUnits;
   for (int lp0 = p0 + warp * kPagesPerTile * kFinTiles; lp0 < p1;
        lp0 += warps * kPagesPerTile * kFinTiles) {
     V mt[kFinTiles][kChunks];
-    V part[kFinTiles][kUnitsPerTile][kChunks];
+    W part[kFinTiles][kChunks][VEC];
 #pragma unroll
     for (int t = 0; t < kFinTiles; ++t) {
       const int lpt = lp0 + t * kPagesPerTile;
-      const bool live = lpt < min(np, p1);
+      const bool live = lpt < min(np, p1);  // tiles past the prefix were never written
       const int tile = lpt * PAGE / tc::kBN;
 #pragma unroll
       for (int c = 0; c < kChunks; ++c) {
-        if (live) {
-          mt[t][c] = load(mt_head + (size_t)tile * BG, c);
+        const int row0 = VEC * lane + 32 * VEC * c;
+        if (live && row0 < BG) {
+          mt[t][c] = *reinterpret_cast<const V *>(mt_head + (size_t)tile * BG + row0);
         } else {
           memset(&mt[t][c], 0, sizeof(V));
         }
 #pragma unroll
-        for (int u = 0; u < kUnitsPerTile; ++u) {
-          if (live && lpt + u / U::kPerPage < np) {
-            part[t][u][c] = load(pp_head + ((size_t)lpt * U::kPerPage + u) * BG, c);
+        for (int e = 0; e < VEC; ++e) {
+          if (live && row0 + e < BG) {
+            part[t][c][e] = *reinterpret_cast<const W *>(pp_head + ((size_t)tile * BG + row0 + e) * kUnits);
           } else {
-            memset(&part[t][u][c], 0, sizeof(V));
+            memset(&part[t][c][e], 0, sizeof(W));
           }
         }
       }
@@ -362,31 +384,33 @@ __device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &p
 #pragma unroll
     for (int t = 0; t < kFinTiles; ++t) {
       const int lpt = lp0 + t * kPagesPerTile;
-      float acc[kUnitsPerTile];
+      float acc[kUnits];
 #pragma unroll
-      for (int u = 0; u < kUnitsPerTile; ++u) acc[u] = 0.f;
+      for (int u = 0; u < kUnits; ++u) acc[u] = 0.f;
 #pragma unroll
       for (int c = 0; c < kChunks; ++c)
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
           const float f = rl[c][e] > 0.f ? exp2f(lanes(mt[t][c], e) - rm[c][e]) * rl[c][e] : 0.f;
 #pragma unroll
-          for (int u = 0; u < kUnitsPerTile; ++u) acc[u] += lanes(part[t][u][c], e) * f;
+          for (int u = 0; u < kUnits; ++u) acc[u] = fmaf(units(part[t][c][e], u), f, acc[u]);
         }
+      float pv[kPagesPerTile];
 #pragma unroll
       for (int pi = 0; pi < kPagesPerTile; ++pi) {
-        float v = 0.f;
+        pv[pi] = 0.f;
 #pragma unroll
-        for (int u = pi * U::kPerPage; u < (pi + 1) * U::kPerPage; ++u) v += acc[u];
-        v = warp_sum(v) * inv_bg;
-        if (lane == 0 && lpt + pi < p1) a.scores[sh_idx * sh.max_pages + lpt + pi] = v;
+        for (int u = pi * U::kPerPage; u < (pi + 1) * U::kPerPage; ++u) pv[pi] += acc[u];
       }
+      const float v = warp_sum_multi<kPagesPerTile>(pv, lane) * inv_bg;
+      const int pi = lane / (32 / kPagesPerTile);
+      if (lane % (32 / kPagesPerTile) == 0 && lpt + pi < p1) a.scores[sh_idx * sh.max_pages + lpt + pi] = v;
     }
   }
 }
 
 template <int D, int PAGE>
-__global__ void __launch_bounds__(kFinThreads) select_finalize(const __grid_constant__ PartialParams pp) {
+__global__ void __launch_bounds__(kFinThreads, 2) select_finalize(const __grid_constant__ PartialParams pp) {
   __shared__ float sM[256], sLinv[256];
   const Shape &sh = pp.sh;
   const SelectPlan &plan = pp.plan;
@@ -404,12 +428,13 @@ __global__ void __launch_bounds__(kFinThreads) select_finalize(const __grid_cons
   if ((int)blockIdx.x < score_ctas) {
     const int p0 = blockIdx.x * plan.fin_pages;  // a multiple of 64 tokens
     const int p1 = min(sh.max_pages, p0 + plan.fin_pages);
+    // (kFinTiles: 64-token tiles whose loads a warp has in flight at once)
     if (sh.BG % 4 == 0) {
-      if (sh.BG <= 128) page_scores<PAGE, 4, 1>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
-      else page_scores<PAGE, 4, 2>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
+      if (sh.BG <= 128) page_scores<PAGE, 4, 1, 4>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
+      else page_scores<PAGE, 4, 2, 2>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
     } else {
-      if (sh.BG <= 32) page_scores<PAGE, 1, 1>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
-      else page_scores<PAGE, 1, 8>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
+      if (sh.BG <= 32) page_scores<PAGE, 1, 1, 4>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
+      else page_scores<PAGE, 1, 8, 1>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
     }
   } else {
     // o_out row: lane j holds the weight 2^(m_j - M) of split j (0 for an empty
@@ -688,15 +713,18 @@ SelectPlan plan_select(const Shape &sh, int num_sms) {
   auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
   size_t off = 4096;  // status word and counters
   const size_t shn = (size_t)sh.S * sh.Hkv;
-  // score CTAs of the finalize pass: about two per SM, each a multiple of 8 tiles
+  // finalize: two resident CTAs per SM and a single wave; the output CTAs take
+  // their share, the score CTAs the rest, each a multiple of 8 tiles (one per warp)
   const long long all_pages = (long long)sh.S * sh.Hkv * sh.max_pages;
-  long long fp = (all_pages + 2LL * num_sms - 1) / (2LL * num_sms);
+  const long long o_ctas = (long long)sh.S * sh.Hkv * ((sh.BG + kRowsPerFinCta - 1) / kRowsPerFinCta);
+  const long long score_target = std::max<long long>(num_sms, 2LL * num_sms - o_ctas);
+  const long long fp = (all_pages + score_target - 1) / score_target;
   const long long tile_pages = tc::kBN / sh.P;  // score CTAs start on tile boundaries
   p.fin_pages = (int)std::max(tile_pages * 8, (fp + tile_pages * 8 - 1) / (tile_pages * 8) * (tile_pages * 8));
   p.off_part_o = off;   off = align(off + shn * p.splits * sh.BG * sh.d * 4);
   p.off_part_ml = off;  off = align(off + shn * p.splits * sh.BG * 2 * 4);
-  const size_t units_per_page = sh.P > tc::kHalfBN ? (size_t)sh.P / tc::kHalfBN : 1;
-  p.off_pagepart = off; off = align(off + shn * sh.max_pages * units_per_page * sh.BG * 4);
+  const size_t units_per_tile = (size_t)tc::kBN / std::min(sh.P, tc::kHalfBN);
+  p.off_pagepart = off; off = align(off + shn * p.max_tiles * sh.BG * units_per_tile * 4);
   p.off_mtile = off;    off = align(off + shn * p.max_tiles * sh.BG * 4);
   p.off_scores = off;   off = align(off + shn * sh.max_pages * 4);
   p.total = off;

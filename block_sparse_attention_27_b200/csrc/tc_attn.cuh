@@ -236,6 +236,13 @@ struct Engine {
           if (!mbar_wait(kv_full(st), (k / STAGES) & 1, ctx)) return false;
           if (k == 0) DSA_TRACE_EVENT(3);
           if (k >= 4 && !mbar_wait(s_free(sb), (((k >> 1) - 2) >> 1) & 1, ctx)) return false;
+          // the buffer still holds P of tile k - 4, which PV(k - 4) reads from TMEM:
+          // that MMA must have completed (not only been issued) before S(k) lands
+          // there.  S(k) is issued at the top of iteration k - kLook, after PV of
+          // tile k - 2 * ((kLook + 2) / 2), the latest PV of this group so far
+          // (k - 4 or later): waiting for that one, whose pv_done phase is the
+          // current one, covers PV(k - 4) (commits complete in order).
+          if (k >= 4 && !mbar_wait(pv_done(k & 1), ((k >> 1) - (kLook + 2) / 2) & 1, ctx)) return false;
           tc_fence_after();
           const uint32_t sk = stage_k(st);
 #pragma unroll
@@ -318,8 +325,10 @@ struct Engine {
         const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * pol.sl2;
         if (tr) DSA_TRACE_EVENT(19);
         // PV of this group's previous tile must have landed before O is rescaled.
-        // (P goes into this tile's own S buffer, whose last reader, PV of the tile
-        // four earlier, was issued before this tile's S and hence is done.)
+        // It is the only PV of the group that may still run here (the one before
+        // completed before this tile's S was issued), so the parity wait below is
+        // unambiguous.  P goes into this tile's own S buffer, whose last reader,
+        // PV of the tile four earlier, has completed for the same reason.
         const bool need = tmax > m_used + kRescaleLog2 || (m_used == -INFINITY && tmax > -INFINITY);
         if (__any_sync(0xffffffffu, need)) {
           float alpha = 1.f;
@@ -384,7 +393,12 @@ struct Engine {
         if (k >= num_tiles - 2 && lead && g == ((num_tiles - 1) & 1)) DSA_TRACE_EVENT(5);
       }
       if (alive && mine > 0) {  // the group's last PV has landed in its O
-        alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 1) & 1, ctx));
+        // Up to two of the group's PVs may still run (the last one and the one
+        // before; older ones completed before the S of a later tile was issued).
+        // A parity wait only tells the current phase from the one before, so
+        // wait for them in order.
+        if (mine >= 2) alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 2) & 1, ctx));
+        if (alive) alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 1) & 1, ctx));
         if (alive) tc_fence_after();
         if (r == 0 && g == ((num_tiles - 1) & 1)) DSA_TRACE_EVENT(6);
       }

@@ -157,3 +157,38 @@ def test_deterministic(dsa_mod):
     b = (dw.idx.clone(), dw.o_sel.clone(), dw.sparse(q, bk, bv).clone())
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def _poison(dsa_mod, ws):
+    """Fill a workspace with 0xFF bytes (NaN as fp32), then zero its status header:
+    a kernel that reads a word it did not write this call now sees NaN."""
+    ws.buf.fill_(0xFF)
+    rc = dsa_mod.load().dsa_workspace_init(dsa_mod._ptr(ws.buf), ws.nbytes, dsa_mod._stream(None))
+    assert rc == dsa_mod.DSA_OK
+
+
+def test_repeatable_on_poisoned_workspaces(dsa_mod):
+    """Full-size 128K: four selection passes and four sparse steps, each on freshly
+    poisoned workspaces, give finite results that are bitwise identical from run to
+    run (catches reads of unwritten workspace and timing-dependent races)."""
+    w = W.make("128k", 0)
+    dw = dsa_mod.DeviceWorkload(w)
+    q, bk, bv = (x.cuda() for x in w.step_inputs(2))
+    first = None
+    for _ in range(4):
+        _poison(dsa_mod, dw.ws_sel)
+        _poison(dsa_mod, dw.ws_sp)
+        idx, cnt, o_sel = (t.clone() for t in dw.select())
+        o_sp = dw.sparse(q, bk, bv).clone()
+        torch.cuda.synchronize()
+        assert dw.ws_sel.status() == dsa_mod.DSA_OK and dw.ws_sp.status() == dsa_mod.DSA_OK
+        bad_sel = (~torch.isfinite(o_sel.float())).nonzero()
+        bad_sp = (~torch.isfinite(o_sp.float())).nonzero()
+        assert len(bad_sel) == 0, f"selection output: {len(bad_sel)} non-finite, first {bad_sel[:4].tolist()}"
+        assert len(bad_sp) == 0, f"sparse output: {len(bad_sp)} non-finite, first {bad_sp[:4].tolist()}"
+        got = (idx, cnt, o_sel, o_sp)
+        if first is None:
+            first = got
+        else:
+            for a, b in zip(first, got):
+                assert torch.equal(a, b)
