@@ -2,6 +2,7 @@
 // layout, launches.  No allocation, no synchronisation (except dsa_get_status).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -47,14 +48,23 @@ int make_shape(const dsa_dims *dims, Shape *out) {
   const int G = d.Hq / d.Hkv;
   if ((long long)d.B * G > 256) return DSA_ERR_UNSUPPORTED;
   if ((long long)d.max_pages * d.page > (1LL << 30)) return DSA_ERR_UNSUPPORTED;
+  if (d.sm_limit < 0) return DSA_ERR_INVALID_ARG;
   Shape s{};
   s.S = d.S; s.B = d.B; s.Hq = d.Hq; s.Hkv = d.Hkv; s.G = G; s.BG = d.B * G;
   s.d = d.d; s.P = d.page; s.max_pages = d.max_pages; s.kmax = d.kmax;
   s.n_phys = d.n_phys;
   s.page_table = d.page_table;
   s.sl2 = (float)(1.4426950408889634 / std::sqrt((double)d.d));
+  s.sm_limit = d.sm_limit;
   *out = s;
   return DSA_OK;
+}
+
+// SMs the selection pass plans for: the device's, or fewer when the caller sets
+// a budget so that it runs beside other work
+int select_sms(const Shape &sh) {
+  const int n = num_sms_current();
+  return sh.sm_limit > 0 ? std::min(n, sh.sm_limit) : n;
 }
 
 template <class T>
@@ -121,7 +131,7 @@ const char *dsa_strerror(int code) {
 size_t dsa_select_workspace_size(const dsa_dims *dims) {
   Shape sh;
   if (make_shape(dims, &sh) != DSA_OK) return 0;
-  return dsa::plan_select(sh, num_sms_current()).total;
+  return dsa::plan_select(sh, select_sms(sh)).total;
 }
 
 size_t dsa_sparse_workspace_size(const dsa_dims *dims) {
@@ -167,7 +177,7 @@ int dsa_select(const void *q_blk, const void *k_cache, const void *v_cache,
   if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o_out) ||
       !aligned16(workspace))
     return DSA_ERR_INVALID_ARG;
-  const dsa::SelectPlan plan = dsa::plan_select(sh, num_sms_current());
+  const dsa::SelectPlan plan = dsa::plan_select(sh, select_sms(sh));
   if (ws_bytes < plan.total) return DSA_ERR_WORKSPACE_TOO_SMALL;
   dsa::SelectArgs a{};
   a.q = static_cast<const __nv_bfloat16 *>(q_blk);
@@ -203,7 +213,7 @@ int dsa_select_static_scratch(const void *q_blk, const void *k_cache, const void
   if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o_out) ||
       (reinterpret_cast<uintptr_t>(status) & 3u) != 0)
     return DSA_ERR_INVALID_ARG;
-  const dsa::SelectPlan plan = dsa::plan_select(sh, num_sms_current());
+  const dsa::SelectPlan plan = dsa::plan_select(sh, select_sms(sh));
   if (plan.total > DSA_SELECT_STATIC_SCRATCH_BYTES) return DSA_ERR_SCRATCH_LIMIT;
   void *scratch = static_scratch_current();
   if (scratch == nullptr) return DSA_ERR_CUDA;

@@ -15,6 +15,7 @@ struct Shape {
   long long n_phys;
   const int32_t *page_table;  // may be null (identity)
   float sl2;                  // log2(e) / sqrt(d)
+  int sm_limit;               // selection pass: SMs it may hold (0 = all)
 };
 
 // TMA map of a paged cache [n_phys, Hkv, P, D] viewed as rows of D bf16; boxes of

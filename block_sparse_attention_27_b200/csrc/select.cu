@@ -330,7 +330,7 @@ __device__ __forceinline__ float warp_sum_multi(const float (&v)[kP], int lane) 
 template <int PAGE, int VEC, int kChunks, int kFinTiles>
 __device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &plan,
                                             const SelectArgs &a, size_t sh_idx, int np, int p0,
-                                            int p1, const float *sM, const float *sLinv) {
+                                            int p1, float *sM, float *sLinv) {
   using U = tc::Units<PAGE>;
   using V = typename std::conditional<VEC == 4, float4, float>::type;
   constexpr int kPagesPerTile = tc::kBN / PAGE;
@@ -339,25 +339,17 @@ __device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &p
   static_assert(kUnits == 4 || kUnits == 2, "units per tile");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int BG = sh.BG;
-  float rm[kChunks][VEC], rl[kChunks][VEC];
-#pragma unroll
-  for (int c = 0; c < kChunks; ++c)
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const int row = VEC * lane + 32 * VEC * c + e;
-      rm[c][e] = row < BG ? sM[row] : 0.f;
-      rl[c][e] = row < BG ? sLinv[row] : 0.f;  // 0: the row does not exist
-    }
   auto lanes = [](const V &v, int e) -> float { return reinterpret_cast<const float *>(&v)[e]; };
   auto units = [](const W &w, int u) -> float { return reinterpret_cast<const float *>(&w)[u]; };
   const float inv_bg = 1.f / (float)BG;
   const int warps = (int)blockDim.x / 32;
+  const int stride = warps * kPagesPerTile * kFinTiles;
   const float *mt_head = a.mtile + sh_idx * plan.max_tiles * BG;
   const float *pp_head = a.pagepart + sh_idx * plan.max_tiles * BG * kUnits;
-  for (int lp0 = p0 + warp * kPagesPerTile * kFinTiles; lp0 < p1;
-       lp0 += warps * kPagesPerTile * kFinTiles) {
-    V mt[kFinTiles][kChunks];
-    W part[kFinTiles][kChunks][VEC];
+  V mt[kFinTiles][kChunks];
+  W part[kFinTiles][kChunks][VEC];
+  // every load of the kFinTiles tiles from lp0 on, issued together
+  auto load = [&](int lp0) {
 #pragma unroll
     for (int t = 0; t < kFinTiles; ++t) {
       const int lpt = lp0 + t * kPagesPerTile;
@@ -381,6 +373,21 @@ __device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &p
         }
       }
     }
+  };
+  int lp0 = p0 + warp * kPagesPerTile * kFinTiles;
+  if (lp0 < p1) load(lp0);  // in flight while the row statistics are formed
+  merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv);
+  __syncthreads();
+  float rm[kChunks][VEC], rl[kChunks][VEC];
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const int row = VEC * lane + 32 * VEC * c + e;
+      rm[c][e] = row < BG ? sM[row] : 0.f;
+      rl[c][e] = row < BG ? sLinv[row] : 0.f;  // 0: the row does not exist
+    }
+  for (; lp0 < p1; lp0 += stride) {
 #pragma unroll
     for (int t = 0; t < kFinTiles; ++t) {
       const int lpt = lp0 + t * kPagesPerTile;
@@ -406,6 +413,7 @@ __device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &p
       const int pi = lane / (32 / kPagesPerTile);
       if (lane % (32 / kPagesPerTile) == 0 && lpt + pi < p1) a.scores[sh_idx * sh.max_pages + lpt + pi] = v;
     }
+    if (lp0 + stride < p1) load(lp0 + stride);
   }
 }
 
@@ -421,11 +429,9 @@ __global__ void __launch_bounds__(kFinThreads, 2) select_finalize(const __grid_c
   const size_t sh_idx = (size_t)s * sh.Hkv + h;
   const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status, false);
   const int np = (n + PAGE - 1) / PAGE;
-  merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv);
-  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int score_ctas = (sh.max_pages + plan.fin_pages - 1) / plan.fin_pages;
-  if ((int)blockIdx.x < score_ctas) {
+  if ((int)blockIdx.x < score_ctas) {  // (page_scores forms the row statistics itself)
     const int p0 = blockIdx.x * plan.fin_pages;  // a multiple of 64 tokens
     const int p1 = min(sh.max_pages, p0 + plan.fin_pages);
     // (kFinTiles: 64-token tiles whose loads a warp has in flight at once)
@@ -437,6 +443,8 @@ __global__ void __launch_bounds__(kFinThreads, 2) select_finalize(const __grid_c
       else page_scores<PAGE, 1, 8, 1>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
     }
   } else {
+    merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv);
+    __syncthreads();
     // o_out row: lane j holds the weight 2^(m_j - M) of split j (0 for an empty
     // split, whose O was never written); kFinBatch splits' O loads are in flight
     // together

@@ -44,7 +44,8 @@ class dsa_dims(ctypes.Structure):
     _fields_ = [("S", ctypes.c_int32), ("B", ctypes.c_int32), ("Hq", ctypes.c_int32),
                 ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("page", ctypes.c_int32),
                 ("max_pages", ctypes.c_int32), ("kmax", ctypes.c_int32),
-                ("n_phys", ctypes.c_int64), ("page_table", ctypes.c_void_p)]
+                ("n_phys", ctypes.c_int64), ("page_table", ctypes.c_void_p),
+                ("sm_limit", ctypes.c_int32)]
 
 
 _lib = None
@@ -104,17 +105,18 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table=None) -> dsa_dims:
+def make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table=None,
+              sm_limit=0) -> dsa_dims:
     return dsa_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys,
-                    None if page_table is None else page_table.data_ptr())
+                    None if page_table is None else page_table.data_ptr(), int(sm_limit))
 
 
-def dims_for(q_blk, k_cache, max_pages, kmax, page_table=None) -> dsa_dims:
+def dims_for(q_blk, k_cache, max_pages, kmax, page_table=None, sm_limit=0) -> dsa_dims:
     S, B, Hq, d = q_blk.shape
     n_phys, Hkv, page, d2 = k_cache.shape
     if d2 != d:
         raise ValueError("q_blk and k_cache disagree on the head dimension")
-    return make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table)
+    return make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table, sm_limit)
 
 
 def _check(t, name, dtype, ndim=None):
@@ -217,7 +219,7 @@ def dsa_sparse_attn(q_blk, k_cache, v_cache, idx, blk_k, blk_v, o_out, stream=No
 class DeviceWorkload:
     """A workload's tensors on the GPU plus the dims, outputs and workspaces of both passes."""
 
-    def __init__(self, w, device="cuda"):
+    def __init__(self, w, device="cuda", sm_limit=0):
         self.w = w
         dev = torch.device(device)
         self.q1 = w.q1.to(dev)
@@ -228,7 +230,7 @@ class DeviceWorkload:
         self.n_ctx = w.n_ctx.to(dev)
         self.topk = w.topk.to(dev)
         self.page_table = None if w.page_table is None else w.page_table.to(dev)
-        self.dims = dims_for(self.q1, self.k_cache, w.max_pages, w.kmax, self.page_table)
+        self.dims = dims_for(self.q1, self.k_cache, w.max_pages, w.kmax, self.page_table, sm_limit)
         S, Hkv = w.S, w.Hkv
         self.idx = torch.full((S, Hkv, w.kmax), -1, dtype=torch.int32, device=dev)
         self.cnt = torch.zeros((S, Hkv), dtype=torch.int32, device=dev)

@@ -89,6 +89,10 @@ typedef struct dsa_dims {
   int32_t kmax;       /* length of an idx row: selected pages per (sequence, KV head), upper bound */
   int64_t n_phys;     /* physical pages held by k_cache / v_cache */
   const int32_t *page_table; /* device [S, max_pages] or NULL (identity) */
+  int32_t sm_limit;   /* selection pass: the most SMs its attention kernel may hold at once,
+                         so that it can run on its own stream beside the sparse steps
+                         (which then keep the other SMs); 0 = every SM of the device.
+                         Workspace sizes depend on it: query them with the same dims. */
 } dsa_dims;
 
 /* cudaStream_t without including the CUDA headers. */

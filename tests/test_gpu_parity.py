@@ -43,8 +43,8 @@ def kp_list(w):
     return [int(w.topk[s]) // w.P for s in range(w.S)]
 
 
-def run_case(dsa_mod, w, steps=(2,)):
-    dw = dsa_mod.DeviceWorkload(w)
+def run_case(dsa_mod, w, steps=(2,), sm_limit=0):
+    dw = dsa_mod.DeviceWorkload(w, sm_limit=sm_limit)
     dw.select()
     torch.cuda.synchronize()
     assert dw.ws_sel.status() == dsa_mod.DSA_OK
@@ -70,6 +70,13 @@ def run_case(dsa_mod, w, steps=(2,)):
 def test_parity(dsa_mod, case):
     name, kw = CASES[case]
     run_case(dsa_mod, W.make(name, 0, **kw), steps=(2, 3))
+
+
+@pytest.mark.parametrize("name,sm_limit", [("8k", 20), ("8k", 37), ("ragged_paged", 6)])
+def test_parity_with_sm_limit(dsa_mod, name, sm_limit):
+    """A selection pass held to fewer SMs (fewer splits) computes the same result."""
+    wname, kw = CASES[name]
+    run_case(dsa_mod, W.make(wname, 0, **kw), sm_limit=sm_limit)
 
 
 @pytest.mark.parametrize("name", ["128k", "batched"])
