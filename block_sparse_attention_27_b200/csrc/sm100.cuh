@@ -117,6 +117,16 @@ __device__ __forceinline__ void cluster_sync() {
                    : "memory");
 }
 // Split form: every thread arrives once (release) and later waits once (acquire).
+// L2 prefetch hints: no data comes back and nothing is ordered by them, so they
+// may name memory that another kernel is still writing.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+// `bytes` (a multiple of 16) from a 16-byte aligned address.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialisation may start while the kernel before it on the stream is still
 // running; grid_dep_wait() returns once that kernel has completed and its

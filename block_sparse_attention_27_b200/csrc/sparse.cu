@@ -218,6 +218,44 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   tc::Engine<D, kSpStages> eng;
   eng.setup(smem_raw, pol);
   if (threadIdx.x == 0) DSA_TRACE_EVENT(32);
+  // While the kernel ahead of this one may still run: L2 prefetches of what this
+  // CTA will read.  The page list is read here without any ordering (through L2
+  // only, so that no stale line stays in L1) and serves only as prefetch
+  // addresses, clamped to the cache; everything the computation uses is read
+  // again after grid_dep_wait().  Warp 1 (the MMA issuer, idle until the first
+  // tiles land) and the softmax warps do this, not the producer.
+  if (eng.warp == 1) {
+    const int lane = eng.lane;
+    if (blk_cta) {
+      const __nv_bfloat16 *bk = a.blk_k + ((size_t)s * sh.B * sh.Hkv + h) * D;
+      const __nv_bfloat16 *bv = a.blk_v + ((size_t)s * sh.B * sh.Hkv + h) * D;
+      for (int u = lane; u < sh.B; u += 32) {
+        sm100::prefetch_l2_bulk(bk + (size_t)u * sh.Hkv * D, D * 2);
+        sm100::prefetch_l2_bulk(bv + (size_t)u * sh.Hkv * D, D * 2);
+      }
+    } else {
+      const int e = c * plan.ppc + lane;
+      if (lane < plan.ppc && e < sh.kmax) {
+        const int lp = __ldcg(a.idx + sh_idx * sh.kmax + e);
+        if (lp >= 0 && lp < sh.max_pages) {
+          const long long ph = sh.page_table ? (long long)__ldcg(sh.page_table + (size_t)s * sh.max_pages + lp)
+                                             : (long long)s * sh.max_pages + lp;
+          if (ph >= 0 && ph < sh.n_phys) {
+            const size_t off = ((size_t)ph * sh.Hkv + h) * PAGE * D;
+            sm100::prefetch_l2_bulk(a.k + off, PAGE * D * 2);
+            sm100::prefetch_l2_bulk(a.v + off, PAGE * D * 2);
+          }
+        }
+      }
+    }
+  } else if (eng.warp >= 2) {  // this thread's half of its query row
+    const int row = row_base + eng.row_in_tile();
+    if (row < sh.BG) {
+      const int b = row / sh.G, g = row % sh.G;
+      sm100::prefetch_l2(a.q + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D +
+                         eng.group() * (D / 2));
+    }
+  }
   // everything below may read what the kernel ahead of this one wrote
   sm100::grid_dep_wait();
   sm100::grid_dep_launch_dependents();
