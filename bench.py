@@ -93,7 +93,7 @@ def kernel_source_sha() -> str:
 
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it matches this source."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(f"{kernel}@{workload}")
