@@ -67,6 +67,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
       if (*ctx.abort) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
         *ctx.abort = 1;
+        // the first wait that gave up, for diagnosis: bits 16..23 = the barrier's
+        // shared-memory address / 8 (mod 256), bits 24..31 = the waiting warp
+        const uint32_t site = (((bar >> 3) & 0xffu) << 16) | ((threadIdx.x >> 5) << 24);
+        uint32_t old = *reinterpret_cast<volatile uint32_t *>(ctx.status);
+        while ((old >> 16) == 0u) {
+          const uint32_t seen = atomicCAS(ctx.status, old, old | site);
+          if (seen == old) break;
+          old = seen;
+        }
         raise_status(ctx.status, kStatusTimeout);
         return false;
       }

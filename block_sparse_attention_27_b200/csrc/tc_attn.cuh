@@ -58,7 +58,7 @@ struct Layout {
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffKV = kOffQ + kHalves * kQHalf;
   static constexpr uint32_t kOffBar = kOffKV + STAGES * kStageBytes;
-  static constexpr int kNumBars = 2 * STAGES + 15;  // the last one is the kernel's own
+  static constexpr int kNumBars = 2 * STAGES + 17;  // the last one is the kernel's own
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kOffML = kOffQ;  // [2 groups][128] (m, l), once Q is dead
   static constexpr uint32_t kBytes = kOffMisc + 16;
@@ -86,11 +86,15 @@ struct Engine {
   __device__ __forceinline__ uint32_t kv_empty(int st) const { return bar(STAGES + st); }
   __device__ __forceinline__ uint32_t s_full(int sb) const { return bar(2 * STAGES + sb); }
   __device__ __forceinline__ uint32_t s_free(int sb) const { return bar(2 * STAGES + 4 + sb); }
-  __device__ __forceinline__ uint32_t p_full(int g) const { return bar(2 * STAGES + 8 + g); }
-  __device__ __forceinline__ uint32_t pv_done(int g) const { return bar(2 * STAGES + 10 + g); }
-  __device__ __forceinline__ uint32_t q_full() const { return bar(2 * STAGES + 12); }
-  __device__ __forceinline__ uint32_t drain() const { return bar(2 * STAGES + 13); }
-  __device__ __forceinline__ uint32_t user_bar() const { return bar(2 * STAGES + 14); }
+  // P of a group's m-th tile is announced on p_full(g, m & 1): with two
+  // barriers per group the group can complete at most one phase ahead of the
+  // MMA issuer's wait on a barrier (its next tile on the same barrier needs an
+  // S that the issuer sends only after that wait), so parity waits stay exact
+  __device__ __forceinline__ uint32_t p_full(int g, int m) const { return bar(2 * STAGES + 8 + 2 * g + (m & 1)); }
+  __device__ __forceinline__ uint32_t pv_done(int g) const { return bar(2 * STAGES + 12 + g); }
+  __device__ __forceinline__ uint32_t q_full() const { return bar(2 * STAGES + 14); }
+  __device__ __forceinline__ uint32_t drain() const { return bar(2 * STAGES + 15); }
+  __device__ __forceinline__ uint32_t user_bar() const { return bar(2 * STAGES + 16); }
   // tile k runs on softmax group k % 2 as that group's (k / 2)-th tile, in S buffer
   // 2 * group + (k / 2) % 2
   static __device__ __forceinline__ int s_buf(int k) { return 2 * (k & 1) + ((k >> 1) & 1); }
@@ -129,7 +133,8 @@ struct Engine {
         mbar_init(s_free(sb), kSoftmaxThreads / 2);
       }
       for (int g = 0; g < 2; ++g) {
-        mbar_init(p_full(g), kSoftmaxThreads / 2);
+        mbar_init(p_full(g, 0), kSoftmaxThreads / 2);
+        mbar_init(p_full(g, 1), kSoftmaxThreads / 2);
         mbar_init(pv_done(g), 1);
       }
       mbar_init(q_full(), kSoftmaxThreads);
@@ -263,7 +268,7 @@ struct Engine {
         for (int j = 0; ok && j < num_tiles; ++j) {
           if (j + kLook < num_tiles && !issue_s(j + kLook)) break;
           const int st = j % STAGES, g = j & 1;
-          if (!mbar_wait(p_full(g), (j >> 1) & 1, ctx)) break;
+          if (!mbar_wait(p_full(g, j >> 1), (j >> 2) & 1, ctx)) break;
           if (j == 2) DSA_TRACE_EVENT(14);
           tc_fence_after();
           const uint32_t sv = stage_v(st);
@@ -386,19 +391,17 @@ struct Engine {
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(s_free(sb));
-        mbar_arrive(p_full(g));
+        mbar_arrive(p_full(g, mine));
         if (tr) DSA_TRACE_EVENT(23);
         if (k == 2 && lead) DSA_TRACE_EVENT(13);
         if (k == 4 && lead) DSA_TRACE_EVENT(29);
         if (k >= num_tiles - 2 && lead && g == ((num_tiles - 1) & 1)) DSA_TRACE_EVENT(5);
       }
       if (alive && mine > 0) {  // the group's last PV has landed in its O
-        // Up to two of the group's PVs may still run (the last one and the one
-        // before; older ones completed before the S of a later tile was issued).
-        // A parity wait only tells the current phase from the one before, so
-        // wait for them in order.
-        if (mine >= 2) alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 2) & 1, ctx));
-        if (alive) alive = __all_sync(0xffffffffu, mbar_wait(pv_done(g), (mine - 1) & 1, ctx));
+        // The MMA issuer commits `drain` once, after its last MMA: a one-phase
+        // barrier, unlike pv_done, whose parity cannot tell a group's last PV
+        // from the one before it once either may already have completed.
+        alive = __all_sync(0xffffffffu, mbar_wait(drain(), 0, ctx));
         if (alive) tc_fence_after();
         if (r == 0 && g == ((num_tiles - 1) & 1)) DSA_TRACE_EVENT(6);
       }

@@ -147,7 +147,10 @@ int dsa_workspace_init(void *workspace, size_t ws_bytes, dsa_stream_t stream);
 
 /* Synchronises `stream`, reads the workspace status word and returns DSA_OK or
  * the most severe device-side code recorded since dsa_workspace_init(); the word
- * is left as it is (sticky).  Returns DSA_ERR_CUDA if the read fails. */
+ * is left as it is (sticky).  Returns DSA_ERR_CUDA if the read fails.  After a
+ * DSA_ERR_DEVICE_TIMEOUT, bits 16..31 of the word (read it directly) identify the
+ * first wait that gave up: bits 16..23 its barrier's shared-memory address / 8
+ * (mod 256), bits 24..31 the waiting warp. */
 int dsa_get_status(const void *workspace, dsa_stream_t stream);
 
 /*
