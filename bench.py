@@ -29,6 +29,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -415,6 +416,16 @@ def _run_ours(args, world, rank, local, dsa):
     del e2e_graphs
     h2d, d2h = b.h2d_d2h_bytes()
 
+    # MAGE's central quantity (outside the timed region): recall of the page set in
+    # use at each step against that step's own top-k, for the reused step-1 set
+    # and for a refresh every 8 steps
+    from block_sparse_attention_27_b200 import recall as R
+    dw = dsa.DeviceWorkload(w)
+    qs = [b.host_q[t].cuda() for t in range(T)]
+    rec_reused = R.step_recall(dw, qs)
+    rec_anchor8 = R.step_recall(dw, qs, anchor=8)
+    del dw, qs
+
     if rank != 0:
         return
     sel_b, sp_b = select_bytes(w), sparse_bytes(w)
@@ -455,6 +466,11 @@ def _run_ours(args, world, rank, local, dsa):
         "clocks": clk.summary(),
         "tensor_tflops_select": round(select_flops(w) / (sel_ms * 1e-3) / 1e12, 1),
         "tensor_peak_tflops": tc_peak,
+        "recall": {"what": "mean over (seq, KV head) of |pages in use & step t's exact top-k| / "
+                           "|exact top-k|, steps 2..T, selections by dsa_select",
+                   "reused_step1_mean": round(float(np.mean(rec_reused[1:])), 4),
+                   "reused_step1_min": round(float(np.min(rec_reused[1:])), 4),
+                   "anchor_every_8_mean": round(float(np.mean(rec_anchor8[1:])), 4)},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
