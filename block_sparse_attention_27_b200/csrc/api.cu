@@ -56,6 +56,7 @@ int make_shape(const dsa_dims *dims, Shape *out) {
   s.page_table = d.page_table;
   s.sl2 = (float)(1.4426950408889634 / std::sqrt((double)d.d));
   s.sm_limit = d.sm_limit;
+  s.lse_out = d.lse_out;
   *out = s;
   return DSA_OK;
 }
@@ -108,6 +109,7 @@ int dsa_version(void) { return 100; }
 int dsa_kernels_per_call(int pass) {
   if (pass == 0) return dsa::kSelectLaunches;
   if (pass == 1) return dsa::kSparseLaunches;
+  if (pass == 2) return dsa::kMergeLaunches;
   return DSA_ERR_INVALID_ARG;
 }
 
@@ -233,6 +235,20 @@ int dsa_select_static_scratch(const void *q_blk, const void *k_cache, const void
   a.scores = at<float>(scratch, plan.off_scores);
   a.status = status;  // the caller's word; the array's header bytes stay unused
   if (dsa::launch_select(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+int dsa_merge_attn(const void *o_a, const float *lse_a, const void *o_b, const float *lse_b,
+                   void *o_out, float *lse_out, int64_t rows, int32_t d, dsa_stream_t stream) {
+  if (!o_a || !lse_a || !o_b || !lse_b || !o_out || rows < 0 || d <= 0 || d % 8 != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(o_a) || !aligned16(o_b) || !aligned16(o_out)) return DSA_ERR_INVALID_ARG;
+  if (rows == 0) return DSA_OK;
+  if (dsa::launch_merge(static_cast<const __nv_bfloat16 *>(o_a), lse_a,
+                        static_cast<const __nv_bfloat16 *>(o_b), lse_b,
+                        static_cast<__nv_bfloat16 *>(o_out), lse_out, rows, d,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;
 }

@@ -16,6 +16,7 @@ struct Shape {
   const int32_t *page_table;  // may be null (identity)
   float sl2;                  // log2(e) / sqrt(d)
   int sm_limit;               // selection pass: SMs it may hold (0 = all)
+  float *lse_out;             // optional [S, B, Hq]: each row's log-sum-exp (natural log)
 };
 
 // TMA map of a paged cache [n_phys, Hkv, P, D] viewed as rows of D bf16; boxes of
@@ -36,6 +37,12 @@ cudaError_t make_blk_tensor_map(CUtensorMap *out, const void *base, long long to
 // Kernel launches issued by one dsa_select / dsa_sparse_attn call.
 constexpr int kSelectLaunches = 3;
 constexpr int kSparseLaunches = 1;
+constexpr int kMergeLaunches = 1;
+
+// dsa_merge_attn (merge.cu)
+cudaError_t launch_merge(const __nv_bfloat16 *o_a, const float *lse_a, const __nv_bfloat16 *o_b,
+                         const float *lse_b, __nv_bfloat16 *o_out, float *lse_out, long long rows,
+                         int d, cudaStream_t stream);
 
 // ---- selection pass ----
 struct SelectPlan {

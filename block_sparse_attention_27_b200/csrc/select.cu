@@ -489,11 +489,15 @@ __global__ void __launch_bounds__(kFinThreads, 2) select_finalize(const __grid_c
         }
       }
     }
-    __nv_bfloat16 *dst = a.o_out + (((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g) * D + lane * kPer;
+    const size_t orow = ((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g;
+    __nv_bfloat16 *dst = a.o_out + orow * D + lane * kPer;
 #pragma unroll
     for (int i = 0; i < kPer; i += 2)
       *reinterpret_cast<__nv_bfloat162 *>(dst + i) =
           __floats2bfloat162_rn(acc[i] * sLinv[row], acc[i + 1] * sLinv[row]);
+    // log-sum-exp of the row's scaled logits over the prefix: (M + log2 L) ln 2
+    if (sh.lse_out && lane == 0)
+      sh.lse_out[orow] = sLinv[row] > 0.f ? (Mrow - log2f(sLinv[row])) * 0.6931471805599453f : -INFINITY;
   }
 }
 

@@ -410,6 +410,9 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
     const int grow = row_base + row;
     const int b = grow / sh.G, g = grow % sh.G;
+    if (sh.lse_out && ch == 0)  // the row's log-sum-exp over its key set: (M + log2 L) ln 2
+      sh.lse_out[((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g] =
+          lsum > 0.f ? (mx + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
     uint4 outv;
     uint32_t *po = reinterpret_cast<uint32_t *>(&outv);
 #pragma unroll

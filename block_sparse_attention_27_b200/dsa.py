@@ -31,7 +31,8 @@ DSA_SELECT_STATIC_SCRATCH_BYTES = 16 << 20
 # every symbol include/dsa.h declares
 EXPORTED = ("dsa_select", "dsa_sparse_attn", "dsa_select_workspace_size",
             "dsa_sparse_workspace_size", "dsa_workspace_init", "dsa_get_status",
-            "dsa_strerror", "dsa_kernels_per_call", "dsa_version", "dsa_select_static_scratch")
+            "dsa_strerror", "dsa_kernels_per_call", "dsa_version", "dsa_select_static_scratch",
+            "dsa_merge_attn")
 
 
 class DsaError(RuntimeError):
@@ -45,7 +46,7 @@ class dsa_dims(ctypes.Structure):
                 ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("page", ctypes.c_int32),
                 ("max_pages", ctypes.c_int32), ("kmax", ctypes.c_int32),
                 ("n_phys", ctypes.c_int64), ("page_table", ctypes.c_void_p),
-                ("sm_limit", ctypes.c_int32)]
+                ("sm_limit", ctypes.c_int32), ("lse_out", ctypes.c_void_p)]
 
 
 _lib = None
@@ -67,6 +68,8 @@ def load(path: str = LIB_PATH):
     lib.dsa_select_static_scratch.restype = ci
     lib.dsa_select_static_scratch.argtypes = [vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp,
                                               dims_p, vp, vp]
+    lib.dsa_merge_attn.restype = ci
+    lib.dsa_merge_attn.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int32, vp]
     lib.dsa_sparse_attn.restype = ci
     lib.dsa_sparse_attn.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, dims_p, vp, vp, vp, sz]
     lib.dsa_select_workspace_size.restype = sz
@@ -108,7 +111,17 @@ def _stream(stream):
 def make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table=None,
               sm_limit=0) -> dsa_dims:
     return dsa_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys,
-                    None if page_table is None else page_table.data_ptr(), int(sm_limit))
+                    None if page_table is None else page_table.data_ptr(), int(sm_limit), None)
+
+
+def _with_lse(dims: dsa_dims, lse_out) -> dsa_dims:
+    """dims for one call, with its optional log-sum-exp output (fp32 [S, B, Hq])."""
+    if lse_out is None:
+        return dims
+    _check(lse_out, "lse_out", torch.float32)
+    d = dsa_dims.from_buffer_copy(dims)
+    d.lse_out = lse_out.data_ptr()
+    return d
 
 
 def dims_for(q_blk, k_cache, max_pages, kmax, page_table=None, sm_limit=0) -> dsa_dims:
@@ -153,7 +166,7 @@ def sparse_workspace_size(dims: dsa_dims) -> int:
 
 
 def dsa_select(q_blk, k_cache, v_cache, n_ctx, page, topk, idx_out, o_out, stream=None, *,
-               dims: dsa_dims, cnt_out, workspace: Workspace):
+               dims: dsa_dims, cnt_out, workspace: Workspace, lse_out=None):
     """Selection pass (see include/dsa.h).  All tensors on the GPU; raises DsaError."""
     _check(q_blk, "q_blk", torch.bfloat16, 4)
     _check(k_cache, "k_cache", torch.bfloat16, 4)
@@ -163,6 +176,7 @@ def dsa_select(q_blk, k_cache, v_cache, n_ctx, page, topk, idx_out, o_out, strea
     _check(idx_out, "idx_out", torch.int32)
     _check(o_out, "o_out", torch.bfloat16)
     _check(cnt_out, "cnt_out", torch.int32)
+    dims = _with_lse(dims, lse_out)
     rc = load().dsa_select(_ptr(q_blk), _ptr(k_cache), _ptr(v_cache), _ptr(n_ctx), int(page),
                            _ptr(topk), _ptr(idx_out), _ptr(o_out), _stream(stream),
                            ctypes.byref(dims), _ptr(cnt_out), _ptr(workspace.buf), workspace.nbytes)
@@ -198,7 +212,7 @@ def status_word(status, stream=None) -> int:
 
 
 def dsa_sparse_attn(q_blk, k_cache, v_cache, idx, blk_k, blk_v, o_out, stream=None, *,
-                    dims: dsa_dims, n_ctx, idx_cnt, workspace: Workspace):
+                    dims: dsa_dims, n_ctx, idx_cnt, workspace: Workspace, lse_out=None):
     """Sparse pass (see include/dsa.h).  All tensors on the GPU; raises DsaError."""
     _check(q_blk, "q_blk", torch.bfloat16, 4)
     _check(k_cache, "k_cache", torch.bfloat16, 4)
@@ -209,11 +223,31 @@ def dsa_sparse_attn(q_blk, k_cache, v_cache, idx, blk_k, blk_v, o_out, stream=No
     _check(o_out, "o_out", torch.bfloat16)
     _check(n_ctx, "n_ctx", torch.int32)
     _check(idx_cnt, "idx_cnt", torch.int32)
+    dims = _with_lse(dims, lse_out)
     rc = load().dsa_sparse_attn(_ptr(q_blk), _ptr(k_cache), _ptr(v_cache), _ptr(idx), _ptr(blk_k),
                                 _ptr(blk_v), _ptr(o_out), _stream(stream), ctypes.byref(dims),
                                 _ptr(n_ctx), _ptr(idx_cnt), _ptr(workspace.buf), workspace.nbytes)
     if rc != DSA_OK:
         raise DsaError(rc, "dsa_sparse_attn")
+
+
+def dsa_merge_attn(o_a, lse_a, o_b, lse_b, o_out, lse_out=None, stream=None):
+    """Merge of two attention results over disjoint key sets (see include/dsa.h).
+    o_*: bf16 [..., d] with the same leading shape; lse_*: fp32 over the leading shape."""
+    for t, n in ((o_a, "o_a"), (o_b, "o_b"), (o_out, "o_out")):
+        _check(t, n, torch.bfloat16)
+    for t, n in ((lse_a, "lse_a"), (lse_b, "lse_b")):
+        _check(t, n, torch.float32)
+    if lse_out is not None:
+        _check(lse_out, "lse_out", torch.float32)
+    d = o_a.shape[-1]
+    rows = o_a.numel() // d
+    if o_b.shape != o_a.shape or o_out.shape != o_a.shape or lse_a.numel() != rows or lse_b.numel() != rows:
+        raise ValueError("dsa_merge_attn: shapes disagree")
+    rc = load().dsa_merge_attn(_ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b), _ptr(o_out),
+                               _ptr(lse_out), rows, d, _stream(stream))
+    if rc != DSA_OK:
+        raise DsaError(rc, "dsa_merge_attn")
 
 
 class DeviceWorkload:
@@ -239,15 +273,16 @@ class DeviceWorkload:
         self.ws_sel = Workspace(select_workspace_size(self.dims), dev)
         self.ws_sp = Workspace(sparse_workspace_size(self.dims), dev)
 
-    def select(self, q=None, stream=None):
+    def select(self, q=None, stream=None, lse_out=None):
         dsa_select(self.q1 if q is None else q, self.k_cache, self.v_cache, self.n_ctx,
                    self.w.P, self.topk, self.idx, self.o_sel, stream, dims=self.dims,
-                   cnt_out=self.cnt, workspace=self.ws_sel)
+                   cnt_out=self.cnt, workspace=self.ws_sel, lse_out=lse_out)
         return self.idx, self.cnt, self.o_sel
 
-    def sparse(self, q, blk_k, blk_v, idx=None, cnt=None, stream=None, out=None):
+    def sparse(self, q, blk_k, blk_v, idx=None, cnt=None, stream=None, out=None, lse_out=None):
         o = self.o_sp if out is None else out
         dsa_sparse_attn(q, self.k_cache, self.v_cache, self.idx if idx is None else idx, blk_k,
                         blk_v, o, stream, dims=self.dims, n_ctx=self.n_ctx,
-                        idx_cnt=self.cnt if cnt is None else cnt, workspace=self.ws_sp)
+                        idx_cnt=self.cnt if cnt is None else cnt, workspace=self.ws_sp,
+                        lse_out=lse_out)
         return o

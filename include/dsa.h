@@ -93,6 +93,10 @@ typedef struct dsa_dims {
                          so that it can run on its own stream beside the sparse steps
                          (which then keep the other SMs); 0 = every SM of the device.
                          Workspace sizes depend on it: query them with the same dims. */
+  float *lse_out;     /* optional device fp32 [S, B, Hq], NULL = not written: the call that
+                         receives these dims stores, per query row, the natural log of the sum
+                         of exp(q.k / sqrt(d)) over the keys it attends to (-inf for none),
+                         so that two attention results can be merged (dsa_merge_attn). */
 } dsa_dims;
 
 /* cudaStream_t without including the CUDA headers. */
@@ -199,11 +203,27 @@ int dsa_select_static_scratch(const void *q_blk, const void *k_cache, const void
                               int32_t *idx_out, void *o_out, dsa_stream_t stream,
                               const dsa_dims *dims, int32_t *cnt_out, uint32_t *status);
 
+/*
+ * Merge of two softmax-attention results over disjoint key sets into the result
+ * over their union.  Not a step of the MAGE page's method: it gives the exact
+ * step-1 output (prefix and block), from the selection pass's prefix-only
+ * output and the sparse pass run with idx_cnt = 0 (the block alone), both with
+ * dims.lse_out set.  For each of `rows` rows:
+ *   lse = log(exp(lse_a) + exp(lse_b)),
+ *   o_out = exp(lse_a - lse) * o_a + exp(lse_b - lse) * o_b,
+ * with o_out = 0 and lse = -inf where both are -inf.  o_a, o_b, o_out: device bf16
+ * [rows, d], 16-byte aligned; lse_a, lse_b: device fp32 [rows]; lse_out: device fp32
+ * [rows] or NULL; d a positive multiple of 8.  o_out may alias o_a or o_b.  One
+ * kernel launch on `stream`; returns DSA_OK or DSA_ERR_INVALID_ARG / DSA_ERR_CUDA.
+ */
+int dsa_merge_attn(const void *o_a, const float *lse_a, const void *o_b, const float *lse_b,
+                   void *o_out, float *lse_out, int64_t rows, int32_t d, dsa_stream_t stream);
+
 /* Static description of a status code. */
 const char *dsa_strerror(int code);
 
 /* Number of kernel launches one call issues on its stream: pass 0 = dsa_select,
- * pass 1 = dsa_sparse_attn (DSA_ERR_INVALID_ARG otherwise).  Useful when
+ * pass 1 = dsa_sparse_attn, pass 2 = dsa_merge_attn (DSA_ERR_INVALID_ARG otherwise).  Useful when
  * capturing calls into a CUDA graph or counting launches. */
 int dsa_kernels_per_call(int pass);
 

@@ -120,3 +120,13 @@ def test_static_scratch_entry_checks_on_host(lib):
                                        ok, ok)
     assert rc == dsa.DSA_ERR_SCRATCH_LIMIT
     assert "static" in dsa.strerror(dsa.DSA_ERR_SCRATCH_LIMIT)
+
+
+def test_merge_entry_checks_on_host(lib):
+    ok = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    assert lib.dsa_merge_attn(ok, ok, ok, ok, ok, None, 0, 128, None) == dsa.DSA_OK  # nothing to do
+    assert lib.dsa_merge_attn(None, ok, ok, ok, ok, None, 4, 128, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_merge_attn(ok, ok, ok, ok, ok, None, 4, 12, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_merge_attn(ok, ok, bad, ok, ok, None, 4, 128, None) == dsa.DSA_ERR_INVALID_ARG
+    assert dsa.kernels_per_call(2) == 1
