@@ -424,6 +424,20 @@ def _run_ours(args, world, rank, local, dsa):
     qs = [b.host_q[t].cuda() for t in range(T)]
     rec_reused = R.step_recall(dw, qs)
     rec_anchor8 = R.step_recall(dw, qs, anchor=8)
+    # exact step-1 output: what it costs beyond the selection pass (which writes its
+    # row log-sum-exps as well): the block-only sparse pass and the LSE merge
+    lse_sel = torch.empty(w.q1.shape[:3], dtype=torch.float32, device="cuda")
+    lse_blk, lse_all = torch.empty_like(lse_sel), torch.empty_like(lse_sel)
+    no_pages = torch.zeros_like(dw.cnt)
+    o_all = torch.empty_like(dw.o_sel)
+    dw.select(lse_out=lse_sel)
+
+    def exact_extra(_):
+        o_blk = dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1, cnt=no_pages, lse_out=lse_blk)
+        dsa.dsa_merge_attn(dw.o_sel, lse_sel, o_blk, lse_blk, o_all, lse_all)
+    for i in range(3):
+        exact_extra(i)
+    exact_us = 1e3 * timed(exact_extra, 20, torch.cuda.current_stream())
     del dw, qs
 
     if rank != 0:
@@ -471,6 +485,7 @@ def _run_ours(args, world, rank, local, dsa):
                    "reused_step1_mean": round(float(np.mean(rec_reused[1:])), 4),
                    "reused_step1_min": round(float(np.min(rec_reused[1:])), 4),
                    "anchor_every_8_mean": round(float(np.mean(rec_anchor8[1:])), 4)},
+        "exact_step1_extra_us": round(exact_us, 2),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
