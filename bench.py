@@ -378,7 +378,7 @@ def _run_ours(args, world, rank, local, dsa):
     hbm_peak, tc_peak, peak_kind = load_peaks()
     T, L = w.T, args.layers
     step_bytes = L * (select_bytes(w) + (T - 1) * sparse_bytes(w))
-    launches_per_step = L * (dsa.kernels_per_call(0) + (T - 1) * dsa.kernels_per_call(1))
+    launches_per_step = L * (dsa.select_launches(b.dims) + (T - 1) * dsa.kernels_per_call(1))
 
     # initial selection (block 0's indices), eager warm-up of every kernel
     for l in range(L):

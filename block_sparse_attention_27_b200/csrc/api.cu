@@ -130,6 +130,13 @@ const char *dsa_strerror(int code) {
   }
 }
 
+int dsa_select_launches(const dsa_dims *dims) {
+  Shape sh;
+  const int rc = make_shape(dims, &sh);
+  if (rc != DSA_OK) return rc;
+  return dsa::plan_select(sh, select_sms(sh)).launches;
+}
+
 size_t dsa_select_workspace_size(const dsa_dims *dims) {
   Shape sh;
   if (make_shape(dims, &sh) != DSA_OK) return 0;
@@ -195,6 +202,9 @@ int dsa_select(const void *q_blk, const void *k_cache, const void *v_cache,
   a.pagepart = at<float>(workspace, plan.off_pagepart);
   a.mtile = at<float>(workspace, plan.off_mtile);
   a.scores = at<float>(workspace, plan.off_scores);
+  a.cand = at<uint64_t>(workspace, plan.off_cand);
+  a.ccnt = at<int32_t>(workspace, plan.off_ccnt);
+  a.counters = at<uint32_t>(workspace, plan.off_counters);
   a.status = at<uint32_t>(workspace, 0);
   if (dsa::launch_select(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DSA_ERR_CUDA;
@@ -233,7 +243,10 @@ int dsa_select_static_scratch(const void *q_blk, const void *k_cache, const void
   a.pagepart = at<float>(scratch, plan.off_pagepart);
   a.mtile = at<float>(scratch, plan.off_mtile);
   a.scores = at<float>(scratch, plan.off_scores);
-  a.status = status;  // the caller's word; the array's header bytes stay unused
+  a.cand = at<uint64_t>(scratch, plan.off_cand);
+  a.ccnt = at<int32_t>(scratch, plan.off_ccnt);
+  a.counters = at<uint32_t>(scratch, plan.off_counters);
+  a.status = status;  // the caller's word; the array's header holds only the group counters
   if (dsa::launch_select(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;

@@ -34,8 +34,10 @@ cudaError_t make_kv_pages_tensor_map(CUtensorMap *out, const void *base, long lo
 cudaError_t make_blk_tensor_map(CUtensorMap *out, const void *base, long long tokens, int Hkv,
                                 int D);
 
-// Kernel launches issued by one dsa_select / dsa_sparse_attn call.
-constexpr int kSelectLaunches = 3;
+// Kernel launches issued by one dsa_select (when all its (sequence, KV head)
+// groups fit in one co-resident launch; see SelectPlan::launches) and by one
+// dsa_sparse_attn call.
+constexpr int kSelectLaunches = 1;
 constexpr int kSparseLaunches = 1;
 constexpr int kMergeLaunches = 1;
 
@@ -46,24 +48,37 @@ cudaError_t launch_merge(const __nv_bfloat16 *o_a, const float *lse_a, const __n
 
 // ---- selection pass ----
 struct SelectPlan {
-  int rowtiles;         // ceil(BG / 128)
-  int splits;           // key splits per (seq, KV head, row tile)
-  int tiles_per_split;  // 64-token tiles per split
-  int max_tiles;        // ceil(max_pages * P / 64)
-  int fin_pages;        // pages per score CTA of the finalize pass
-  size_t off_part_o, off_part_ml, off_pagepart, off_mtile, off_scores, total;
+  int rowtiles;          // ceil(BG / 128)
+  int splits;            // key splits per (seq, KV head, row tile)
+  int tiles_per_split;   // 64-token tiles per split
+  int max_tiles;         // ceil(max_pages * P / 64)
+  int group_ctas;        // CTAs of one (seq, KV head) group: splits * rowtiles
+  int groups_per_launch; // groups of one co-resident (cooperative) launch
+  int launches;          // ceil(S * Hkv / groups_per_launch)
+  int bgp;               // BG rounded up to a multiple of 4: row stride of pagepart / mtile
+  int slot_len;          // entries of one CTA's candidate list
+  size_t off_counters;   // in the zeroed header: four counters per group of a launch
+  size_t off_part_o, off_part_ml, off_pagepart, off_mtile, off_scores, off_cand, off_ccnt, total;
 };
+
+// Counters of a group (barrier arrivals, candidate hand-offs, output rows taken,
+// CTAs done with output rows): 4 per group, in the workspace header after its
+// first 256 bytes.
+constexpr int kMaxGroupsPerLaunch = 240;
 
 struct SelectArgs {
   const __nv_bfloat16 *q, *k, *v;
   const int32_t *n_ctx, *topk;
   int32_t *idx_out, *cnt_out;
   __nv_bfloat16 *o_out;
-  float *part_o;    // [S, Hkv, rowtiles*splits... ] see select.cu
-  float *part_ml;
-  float *pagepart;  // [S, Hkv, max_pages, BG]
-  float *mtile;     // [S, Hkv, max_tiles, BG]
-  float *scores;    // [S, Hkv, max_pages]
+  float *part_o;      // [S*Hkv][splits][BG][D] unnormalised split outputs
+  float *part_ml;     // [S*Hkv][splits][BG] (m, l) of each split (log2 domain)
+  float *pagepart;    // [S*Hkv][max_tiles][bgp][units per tile]
+  float *mtile;       // [S*Hkv][max_tiles][bgp]
+  float *scores;      // [S*Hkv][max_pages]
+  uint64_t *cand;     // [S*Hkv][group_ctas][slot_len] local candidates (score bits << 32 | ~page)
+  int32_t *ccnt;      // [S*Hkv][group_ctas] candidates of each CTA
+  uint32_t *counters; // [groups_per_launch][4] (arrive, leave, output rows, done)
   uint32_t *status;
 };
 

@@ -3,19 +3,25 @@
 // KV head ("MAGE: All-[MASK] Block Already Knows Where to Look in Block
 // Diffusion LLM", Approach).
 //
-// Three launches on the caller's stream, each a programmatic dependent of the
-// one before it:
-//   1. select_partial: split-KV attention on the tcgen05 engine (tc_attn.cuh).
-//      CTA = (split, 128-row tile) x KV head x sequence, one wave over the SMs;
-//      the split's 64-token tiles stream through a TMA ring.  Per split it
-//      writes the unnormalised output O_j with its row max m_j and sum l_j, and
-//      per (tile, row) the partial probability mass of each unit of the tile
-//      (min(page, 32) keys of one page) relative to the row's reference max at
-//      that tile (pagepart, [tile][row][unit]), together with that max (mtile).
-//   2. select_finalize: merges the splits into o_out and turns the partial
-//      masses into page scores  S_h[q] = (1/BG) sum_rows pagepart * 2^(mtile-M) / L.
-//   3. select_topk: radix select of the kp-th largest score per (seq, KV head),
-//      ties broken towards the lower page index, emitted in ascending order.
+// One kernel, select_fused, launched cooperatively (all its CTAs co-resident).
+// A group is one (sequence, KV head); its CTAs are the (split, 128-row tile)
+// pairs, one wave over the SMs.
+//   1. Split-KV attention on the tcgen05 engine (tc_attn.cuh): the split's
+//      64-token tiles stream through a TMA ring.  Per split the CTA writes the
+//      unnormalised output O_j with its row max m_j and sum l_j, and per (tile,
+//      row) the partial probability mass of each unit of the tile (min(page, 32)
+//      keys of one page) relative to the row's reference max at that tile
+//      (pagepart, [tile][row][unit]), together with that max (mtile).
+//   2. Group barrier: a counter in the workspace header, bounded wait.
+//   3. Every CTA of the group forms each row's global M = max_j m_j and
+//      L = sum_j l_j 2^(m_j - M), writes its share of the rows of o_out, and
+//      turns the partial masses of its share of the pages into page scores
+//        S_h[q] = (1/BG) sum_rows pagepart * 2^(mtile - M) / L,
+//      then keeps its local top-kp pages (radix select, ties to the lower page)
+//      as candidates, in ascending page order.
+//   4. The group's last CTA to finish step 3 selects the kp largest among the
+//      candidates (the global top-kp of the head is among them: each of its
+//      pages is in the local top-kp of its own CTA) and writes them ascending.
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -33,10 +39,11 @@ struct PartialParams {
   Shape sh;
   SelectPlan plan;
   SelectArgs a;
+  int group0;  // first (sequence, KV head) group of this launch: s * Hkv + h
 };
 
 // ---------------------------------------------------------------------------
-// select_partial: tcgen05 split-KV attention (tc_attn.cuh engine) over the
+// Step 1, the engine policy: tcgen05 split-KV attention (tc_attn.cuh) over the
 // split's contiguous 64-token tiles of the prefix, loaded page by page through
 // the page table.  After each tile the softmax threads record, per (page, row),
 // the tile's probability mass relative to the row's reference max (pagepart)
@@ -44,6 +51,16 @@ struct PartialParams {
 // part_ml.
 // ---------------------------------------------------------------------------
 constexpr int kSelStages = 5;
+
+// K/V tiles are read once: loaded with an evict-first L2 policy, so that the
+// partials the tail reads back (written during the loop) stay in L2.
+#ifndef DSA_KV_EVICT_FIRST
+#define DSA_KV_EVICT_FIRST 1
+#endif
+// The partials (written once, read back by the tail) are stored evict-last.
+#ifndef DSA_PART_EVICT_LAST
+#define DSA_PART_EVICT_LAST 1
+#endif
 
 template <int D, int PAGE>
 struct SelectPolicy {
@@ -58,7 +75,8 @@ struct SelectPolicy {
   float *pagepart_head;             // pagepart[s, h, 0, 0, 0]
   uint32_t *status;
   long long n_phys, phys0;          // phys0 = s*max_pages (identity map)
-  int Hkv, h, G, Hq, BG, n, np, t_begin, row_base;
+  int Hkv, h, G, Hq, BG, BGp, n, np, t_begin, row_base;  // BGp: row stride of mtile / pagepart
+  bool report;                      // this CTA reports bad page-table entries (row tile 0)
   float sl2;
 
   __device__ __forceinline__ long long phys_of(int lp) const {
@@ -84,7 +102,7 @@ struct SelectPolicy {
     const int lp0 = (t_begin + k) * tc::kBN / PAGE;
     const long long my = phys_of(lp0 + (lane < kPages ? lane : 0));
     const bool valid = lane < kPages && my >= 0;
-    if (lane < kPages && my < 0 && lp0 + lane < np && blockIdx.x == 0)
+    if (lane < kPages && my < 0 && lp0 + lane < np && report)
       raise_status(status, kStatusBadIndex);
     const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
     const long long p0 = __shfl_sync(0xffffffffu, my, 0);
@@ -92,12 +110,20 @@ struct SelectPolicy {
     const bool run = kPages > 1 && __all_sync(0xffffffffu, consec);
     if (lane == 0)
       sm100::mbar_arrive_expect_tx(bar, (uint32_t)__popc(vmask) * PAGE * 128u * kHalves * 2u);
+#if DSA_KV_EVICT_FIRST
+    const uint64_t l2pol = sm100::l2_policy_evict_first();
+#endif
     if (run) {  // the whole tile in one box per half and tensor
       if (lane < 2 * kHalves) {
         const int hf = lane % kHalves;
         const bool isv = lane >= kHalves;
+#if DSA_KV_EVICT_FIRST
+        sm100::tma_load_4d_hint((isv ? sv : sk) + hf * half_bytes, isv ? vmap4 : kmap4, bar, hf * 64, 0,
+                                h, (int)p0, l2pol);
+#else
         sm100::tma_load_4d((isv ? sv : sk) + hf * half_bytes, isv ? vmap4 : kmap4, bar, hf * 64, 0, h,
                            (int)p0);
+#endif
       }
       return;
     }
@@ -107,8 +133,13 @@ struct SelectPolicy {
       const int hf = rem % kHalves;
       const bool isv = rem >= kHalves;
       const int y = (int)((ph * Hkv + h) * PAGE);
+#if DSA_KV_EVICT_FIRST
+      sm100::tma_load_2d_hint((isv ? sv : sk) + hf * half_bytes + pi * PAGE * 128, isv ? vmap : kmap,
+                              bar, hf * 64, y, l2pol);
+#else
       sm100::tma_load_2d((isv ? sv : sk) + hf * half_bytes + pi * PAGE * 128, isv ? vmap : kmap, bar,
                          hf * 64, y);
+#endif
     }
   }
   __device__ __forceinline__ const __nv_bfloat16 *q_row(int r) const {
@@ -138,113 +169,29 @@ struct SelectPolicy {
     const int row = row_base + r;
     if (row >= BG) return;
     const int tile = t_begin + k;
-    mtile_head[(size_t)tile * BG + row] = m_used;
-    // the row's unit masses of the tile, one vector store (units past the prefix hold 0)
-    float *dst = pagepart_head + ((size_t)tile * BG + row) * U::kPerTile;
+    // the row's tile max and unit masses of the tile, one vector store (units
+    // past the prefix hold 0)
+    float *dst = pagepart_head + ((size_t)tile * BGp + row) * U::kPerTile;
+#if DSA_PART_EVICT_LAST
+    const uint64_t pol = sm100::l2_policy_evict_last();
+    sm100::st_hint(mtile_head + (size_t)tile * BGp + row, m_used, pol);
+    if constexpr (U::kPerTile == 4)
+      sm100::st_hint(reinterpret_cast<float4 *>(dst), make_float4(usum[0], usum[1], usum[2], usum[3]), pol);
+    else
+      sm100::st_hint(reinterpret_cast<float2 *>(dst), make_float2(usum[0], usum[1]), pol);
+#else
+    mtile_head[(size_t)tile * BGp + row] = m_used;
     if constexpr (U::kPerTile == 4)
       *reinterpret_cast<float4 *>(dst) = make_float4(usum[0], usum[1], usum[2], usum[3]);
     else
       *reinterpret_cast<float2 *>(dst) = make_float2(usum[0], usum[1]);
+#endif
   }
 };
 
-template <int D, int PAGE>
-__global__ void __launch_bounds__(tc::kThreads, 1)
-    select_partial(const __grid_constant__ PartialParams pp, const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kmap4,
-                   const __grid_constant__ CUtensorMap vmap4) {
-  extern __shared__ unsigned char smem_raw[];
-  const Shape &sh = pp.sh;
-  const SelectPlan &plan = pp.plan;
-  const SelectArgs &a = pp.a;
-  const int s = blockIdx.z, h = blockIdx.y;
-  const int split = blockIdx.x / plan.rowtiles, rt = blockIdx.x % plan.rowtiles;
-  if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
-  SelectPolicy<D, PAGE> pol;
-  pol.kmap = &kmap;
-  pol.vmap = &vmap;
-  pol.kmap4 = &kmap4;
-  pol.vmap4 = &vmap4;
-  tc::Engine<D, kSelStages> eng;
-  eng.setup(smem_raw, pol);
-  // everything below may read what the kernel ahead of this one wrote
-  sm100::grid_dep_wait();
-  sm100::grid_dep_launch_dependents();
-
-  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status,
-                             threadIdx.x == 0 && blockIdx.x == 0);
-  const int ntiles = (n + tc::kBN - 1) / tc::kBN;
-  const int t_begin = split * plan.tiles_per_split;
-  const int num_tiles = max(0, min(ntiles, t_begin + plan.tiles_per_split) - t_begin);
-  const size_t sh_idx = (size_t)s * sh.Hkv + h;
-  pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
-  pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
-  pol.mtile_head = a.mtile + sh_idx * plan.max_tiles * sh.BG;
-  pol.pagepart_head = a.pagepart + sh_idx * plan.max_tiles * sh.BG * tc::Units<PAGE>::kPerTile;
-  pol.status = a.status;
-  pol.n_phys = sh.n_phys;
-  pol.phys0 = (long long)s * sh.max_pages;
-  pol.Hkv = sh.Hkv;
-  pol.h = h;
-  pol.G = sh.G;
-  pol.Hq = sh.Hq;
-  pol.BG = sh.BG;
-  pol.n = n;
-  pol.np = (n + PAGE - 1) / PAGE;
-  pol.t_begin = t_begin;
-  pol.row_base = rt * kRowsPerCta;
-  pol.sl2 = sh.sl2;
-  eng.init(a.status, pol, num_tiles);
-  float m, l;
-  eng.template run<PAGE>(pol, num_tiles, m, l);
-  float m_row, l_row, wa, wb;
-  eng.finish(m, l, m_row, l_row, wa, wb);
-  if (eng.warp >= 2) {
-    // O = wa * O_0 + wb * O_1 relative to m_row; this thread writes its half of the columns
-    const int g = eng.group();
-    const int row = rt * kRowsPerCta + eng.row_in_tile();
-    const bool row_ok = row < sh.BG;
-    const size_t prow = ((sh_idx * plan.splits + split) * sh.BG + row);
-#pragma unroll
-    for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 32) {
-      uint32_t oa[32], ob[32];
-      eng.load_o(0, c0, oa);
-      eng.load_o(1, c0, ob);
-      if (row_ok && l_row > 0.f) {
-        float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * D + c0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          float v[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = wa > 0.f ? wa * __uint_as_float(oa[4 * i + e]) : 0.f;
-            const float x1 = wb > 0.f ? wb * __uint_as_float(ob[4 * i + e]) : 0.f;
-            v[e] = x0 + x1;
-          }
-          dst[i] = make_float4(v[0], v[1], v[2], v[3]);
-        }
-      }
-    }
-    if (row_ok && g == 0)
-      *reinterpret_cast<float2 *>(a.part_ml + prow * 2) =
-          l_row > 0.f ? make_float2(m_row, l_row) : make_float2(-INFINITY, 0.f);
-    if (row == rt * kRowsPerCta) DSA_TRACE_EVENT(7);
-  }
-  eng.teardown();
-  if (threadIdx.x == 0) DSA_TRACE_EVENT(11);
-}
-
 // ---------------------------------------------------------------------------
-// select_finalize: merges the splits.  Every CTA first forms, for each query
-// row, the global reference M = max_j m_j and 1/L with L = sum_j l_j 2^(m_j - M)
-// (one online pass over the splits).  Score CTAs then turn the partial masses of
-// their pages into  S_h[q] = (1/BG) sum_rows pagepart * 2^(mtile - M) / L;
-// output CTAs write o_out = sum_j 2^(m_j - M) O_j / L in bf16.
+// Steps 3-4 of the tail: the splits' row statistics, page scores, output rows.
 // ---------------------------------------------------------------------------
-constexpr int kFinThreads = 256;
-constexpr int kRowsPerFinCta = 8;   // output CTAs: one query row per warp
-constexpr int kFinBatch = 16;       // output CTAs: split partials a lane loads at once
-
 // Folds a partial (m, l) into the running (M, L) of a row (log2 domain); an
 // empty partial (l = 0) leaves it unchanged.
 __device__ __forceinline__ void merge_ml(float &M, float &L, float m, float l) {
@@ -259,11 +206,13 @@ __device__ __forceinline__ void merge_ml(float &M, float &L, float m, float l) {
 
 // sM[row] = M and sLinv[row] = 1/L over all splits.  Each row gets tpr = the
 // largest power of two <= blockDim.x / BG (at most 32) threads of one warp; each
-// of them loads its splits 8 at a time (all in flight together), then the tpr
-// partial results are combined with shuffles.
+// of them loads its splits 16 at a time (all in flight together), then the tpr
+// partial results are combined with shuffles.  after_issue() runs once, right
+// after the first loads are issued (so that they go ahead of whatever it issues).
+template <class AfterIssue>
 __device__ __forceinline__ void merged_row_stats(const Shape &sh, const SelectPlan &plan,
                                                  const float *part_ml, size_t sh_idx, float *sM,
-                                                 float *sLinv) {
+                                                 float *sLinv, AfterIssue after_issue) {
   int tpr = 1;
   while (tpr < 32 && 2 * tpr * sh.BG <= (int)blockDim.x) tpr *= 2;
   const int sub = threadIdx.x % tpr;
@@ -274,15 +223,16 @@ __device__ __forceinline__ void merged_row_stats(const Shape &sh, const SelectPl
     const int row = row0 + (int)threadIdx.x / tpr;
     const bool valid = row < sh.BG;
     float M = -INFINITY, L = 0.f;
-    for (int j0 = sub; j0 < plan.splits; j0 += 8 * tpr) {
-      float2 v[8];
+    for (int j0 = sub; j0 < plan.splits; j0 += 16 * tpr) {
+      float2 v[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         const int j = j0 + u * tpr;
-        v[u] = (valid && j < plan.splits) ? ml[(size_t)j * sh.BG + row] : make_float2(-INFINITY, 0.f);
+        v[u] = (valid && j < plan.splits) ? __ldcg(&ml[(size_t)j * sh.BG + row]) : make_float2(-INFINITY, 0.f);
       }
+      if (row0 == 0 && j0 == sub) after_issue();  // (the loads above are already issued)
 #pragma unroll
-      for (int u = 0; u < 8; ++u) merge_ml(M, L, v[u].x, v[u].y);
+      for (int u = 0; u < 16; ++u) merge_ml(M, L, v[u].x, v[u].y);
     }
     for (int o = tpr / 2; o > 0; o >>= 1) {
       const float M2 = __shfl_xor_sync(0xffffffffu, M, o);
@@ -322,170 +272,56 @@ __device__ __forceinline__ float warp_sum_multi(const float (&v)[kP], int lane) 
   }
 }
 
-// Page scores of the pages [p0, p1) (tile-aligned) of one (sequence, KV head).
-// Lane i of a warp handles the rows VEC*i + 32*VEC*c + e (c < kChunks, e < VEC):
-// their M and 1/L stay in registers, and for kFinTiles tiles at a time the
-// tile maxima and each row's vector of unit masses are loaded before any of
-// them is used.
-template <int PAGE, int VEC, int kChunks, int kFinTiles>
-__device__ __forceinline__ void page_scores(const Shape &sh, const SelectPlan &plan,
-                                            const SelectArgs &a, size_t sh_idx, int np, int p0,
-                                            int p1, float *sM, float *sLinv) {
-  using U = tc::Units<PAGE>;
-  using V = typename std::conditional<VEC == 4, float4, float>::type;
-  constexpr int kPagesPerTile = tc::kBN / PAGE;
-  constexpr int kUnits = U::kPerTile;  // 4 or 2
-  using W = typename std::conditional<kUnits == 4, float4, float2>::type;
-  static_assert(kUnits == 4 || kUnits == 2, "units per tile");
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int BG = sh.BG;
-  auto lanes = [](const V &v, int e) -> float { return reinterpret_cast<const float *>(&v)[e]; };
-  auto units = [](const W &w, int u) -> float { return reinterpret_cast<const float *>(&w)[u]; };
-  const float inv_bg = 1.f / (float)BG;
-  const int warps = (int)blockDim.x / 32;
-  const int stride = warps * kPagesPerTile * kFinTiles;
-  const float *mt_head = a.mtile + sh_idx * plan.max_tiles * BG;
-  const float *pp_head = a.pagepart + sh_idx * plan.max_tiles * BG * kUnits;
-  V mt[kFinTiles][kChunks];
-  W part[kFinTiles][kChunks][VEC];
-  // every load of the kFinTiles tiles from lp0 on, issued together
-  auto load = [&](int lp0) {
-#pragma unroll
-    for (int t = 0; t < kFinTiles; ++t) {
-      const int lpt = lp0 + t * kPagesPerTile;
-      const bool live = lpt < min(np, p1);  // tiles past the prefix were never written
-      const int tile = lpt * PAGE / tc::kBN;
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
-        const int row0 = VEC * lane + 32 * VEC * c;
-        if (live && row0 < BG) {
-          mt[t][c] = *reinterpret_cast<const V *>(mt_head + (size_t)tile * BG + row0);
-        } else {
-          memset(&mt[t][c], 0, sizeof(V));
-        }
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          if (live && row0 + e < BG) {
-            part[t][c][e] = *reinterpret_cast<const W *>(pp_head + ((size_t)tile * BG + row0 + e) * kUnits);
-          } else {
-            memset(&part[t][c][e], 0, sizeof(W));
-          }
-        }
-      }
-    }
-  };
-  int lp0 = p0 + warp * kPagesPerTile * kFinTiles;
-  if (lp0 < p1) load(lp0);  // in flight while the row statistics are formed
-  merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv);
-  __syncthreads();
-  float rm[kChunks][VEC], rl[kChunks][VEC];
-#pragma unroll
-  for (int c = 0; c < kChunks; ++c)
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      const int row = VEC * lane + 32 * VEC * c + e;
-      rm[c][e] = row < BG ? sM[row] : 0.f;
-      rl[c][e] = row < BG ? sLinv[row] : 0.f;  // 0: the row does not exist
-    }
-  for (; lp0 < p1; lp0 += stride) {
-#pragma unroll
-    for (int t = 0; t < kFinTiles; ++t) {
-      const int lpt = lp0 + t * kPagesPerTile;
-      float acc[kUnits];
-#pragma unroll
-      for (int u = 0; u < kUnits; ++u) acc[u] = 0.f;
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c)
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          const float f = rl[c][e] > 0.f ? exp2f(lanes(mt[t][c], e) - rm[c][e]) * rl[c][e] : 0.f;
-#pragma unroll
-          for (int u = 0; u < kUnits; ++u) acc[u] = fmaf(units(part[t][c][e], u), f, acc[u]);
-        }
-      float pv[kPagesPerTile];
-#pragma unroll
-      for (int pi = 0; pi < kPagesPerTile; ++pi) {
-        pv[pi] = 0.f;
-#pragma unroll
-        for (int u = pi * U::kPerPage; u < (pi + 1) * U::kPerPage; ++u) pv[pi] += acc[u];
-      }
-      const float v = warp_sum_multi<kPagesPerTile>(pv, lane) * inv_bg;
-      const int pi = lane / (32 / kPagesPerTile);
-      if (lane % (32 / kPagesPerTile) == 0 && lpt + pi < p1) a.scores[sh_idx * sh.max_pages + lpt + pi] = v;
-    }
-    if (lp0 + stride < p1) load(lp0 + stride);
-  }
-}
+// One row of o_out (0 <= row < BG of the group), merged by one warp:
+//   o_out = sum_j 2^(m_j - M) O_j / L  (bf16),  lse = (M + log2 L) ln 2.
+// Lane j of the warp loads the (m, l) of split j while kFinBatch splits' O rows
+// are loaded together; an empty split (l = 0, O never written) gets weight 0.
+constexpr int kFinBatch = 20;
 
-template <int D, int PAGE>
-__global__ void __launch_bounds__(kFinThreads, 2) select_finalize(const __grid_constant__ PartialParams pp) {
-  __shared__ float sM[256], sLinv[256];
-  const Shape &sh = pp.sh;
-  const SelectPlan &plan = pp.plan;
-  const SelectArgs &a = pp.a;
-  sm100::grid_dep_wait();  // the partials of select_partial
-  sm100::grid_dep_launch_dependents();
-  const int s = blockIdx.z, h = blockIdx.y;
-  const size_t sh_idx = (size_t)s * sh.Hkv + h;
-  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status, false);
-  const int np = (n + PAGE - 1) / PAGE;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int score_ctas = (sh.max_pages + plan.fin_pages - 1) / plan.fin_pages;
-  if ((int)blockIdx.x < score_ctas) {  // (page_scores forms the row statistics itself)
-    const int p0 = blockIdx.x * plan.fin_pages;  // a multiple of 64 tokens
-    const int p1 = min(sh.max_pages, p0 + plan.fin_pages);
-    // (kFinTiles: 64-token tiles whose loads a warp has in flight at once)
-    if (sh.BG % 4 == 0) {
-      if (sh.BG <= 128) page_scores<PAGE, 4, 1, 4>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
-      else page_scores<PAGE, 4, 2, 2>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
-    } else {
-      if (sh.BG <= 32) page_scores<PAGE, 1, 1, 4>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
-      else page_scores<PAGE, 1, 8, 1>(sh, plan, a, sh_idx, np, p0, p1, sM, sLinv);
-    }
-  } else {
-    merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv);
-    __syncthreads();
-    // o_out row: lane j holds the weight 2^(m_j - M) of split j (0 for an empty
-    // split, whose O was never written); kFinBatch splits' O loads are in flight
-    // together
-    const int row = (blockIdx.x - score_ctas) * kRowsPerFinCta + warp;
-    if (row >= sh.BG) return;
+template <int D>
+__device__ __forceinline__ void merge_output_row(const Shape &sh, const SelectPlan &plan,
+                                                 const SelectArgs &a, size_t sh_idx, int s, int h,
+                                                 int row, const float *sM, const float *sLinv) {
+  static_assert(D / 32 == 4 || D / 32 == 2, "columns per lane");
+  constexpr int kPer = D / 32;
+  using V = typename std::conditional<kPer == 4, float4, float2>::type;
+  const int lane = threadIdx.x & 31;
+  {
     const int b = row / sh.G, g = row % sh.G;
-    static_assert(D / 32 == 4 || D / 32 == 2, "columns per lane");
-    constexpr int kPer = D / 32;
-    using V = typename std::conditional<kPer == 4, float4, float2>::type;
     float acc[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
     const float Mrow = sM[row];
     for (int j0 = 0; j0 < plan.splits; j0 += 32) {
-      float w_lane = 0.f;
+      // lane j: the (m, l) of split j0 + j; its O rows are loaded alongside, and
+      // weighted once the (m, l) are in
+      float2 ml_lane = make_float2(-INFINITY, 0.f);
       if (j0 + lane < plan.splits) {
         const size_t r = (sh_idx * plan.splits + j0 + lane) * sh.BG + row;
-        const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + r * 2);
-        w_lane = ml.y > 0.f ? exp2f(ml.x - Mrow) : 0.f;
+        ml_lane = __ldcg(reinterpret_cast<const float2 *>(a.part_ml + r * 2));
       }
       const int nj = min(32, plan.splits - j0);
       for (int jb = 0; jb < nj; jb += kFinBatch) {
         V o[kFinBatch];
-        float w[kFinBatch];
 #pragma unroll
         for (int u = 0; u < kFinBatch; ++u) {
-          w[u] = __shfl_sync(0xffffffffu, w_lane, (jb + u) & 31);
-          const bool use = jb + u < nj && w[u] > 0.f;
-          if (use) {
+          if (jb + u < nj) {
             const size_t r = (sh_idx * plan.splits + j0 + jb + u) * sh.BG + row;
-            o[u] = *reinterpret_cast<const V *>(a.part_o + r * D + lane * kPer);
+            o[u] = __ldcg(reinterpret_cast<const V *>(a.part_o + r * D + lane * kPer));
           } else {
             memset(&o[u], 0, sizeof(V));
-            w[u] = 0.f;
           }
         }
+        const float w_lane = ml_lane.y > 0.f ? exp2f(ml_lane.x - Mrow) : 0.f;
 #pragma unroll
         for (int u = 0; u < kFinBatch; ++u) {
-          const float *ov = reinterpret_cast<const float *>(&o[u]);
+          // an empty split (weight 0) never wrote its O: its loaded values are not used
+          const float w = __shfl_sync(0xffffffffu, w_lane, (jb + u) & 31);
+          if (jb + u < nj && w > 0.f) {
+            const float *ov = reinterpret_cast<const float *>(&o[u]);
 #pragma unroll
-          for (int i = 0; i < kPer; ++i) acc[i] += w[u] * ov[i];
+            for (int i = 0; i < kPer; ++i) acc[i] += w * ov[i];
+          }
         }
       }
     }
@@ -502,81 +338,47 @@ __global__ void __launch_bounds__(kFinThreads, 2) select_finalize(const __grid_c
 }
 
 // ---------------------------------------------------------------------------
-// select_topk: one CTA per (sequence, KV head).  Page scores are >= 0, so their
-// fp32 bit patterns order like the values; a 4-pass radix select (8 bits per
-// pass, histogram in shared memory, bin search by one warp) finds the kp-th
-// largest key T.  Pages with key > T are kept, and among keys == T the lowest
-// page indices, so ties go to the lower index; an ordered compaction writes the
-// kept pages in ascending order.
+// Block-wide top-k by radix select.  Page scores are >= 0, so their fp32 bit
+// patterns order like the values.  A 4-pass radix select (8 bits per pass,
+// histogram in shared memory, bin search by one warp) finds the take-th largest
+// key T; the keys > T are kept, and among the keys == T the lowest positions.
+// An ordered compaction then emits the kept positions in ascending order, so a
+// list sorted by page keeps ties towards the lower page.
 // ---------------------------------------------------------------------------
-constexpr int kTopkThreads = 1024;
-constexpr int kTopkSmemKeys = 11264;  // keys staged in shared memory up to this many pages (44 KB)
+struct TopkScratch {
+  uint32_t hist[256];
+  uint32_t scan_eq[32], scan_gt[32];
+  uint32_t digit, remaining, flag, bad;
+};
 
 __device__ __forceinline__ uint32_t score_key(float v) {
-  return v > 0.f ? __float_as_uint(v) : 0u;  // -0 folds onto +0
+  return v > 0.f ? __float_as_uint(v) : 0u;  // -0 (and NaN, reported separately) fold onto +0
 }
 
-__global__ void __launch_bounds__(kTopkThreads) select_topk(const __grid_constant__ PartialParams pp) {
-  __shared__ uint32_t keys[kTopkSmemKeys];
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_digit, s_remaining;
-  __shared__ uint32_t scan_eq[kTopkThreads / 32], scan_gt[kTopkThreads / 32];
-  __shared__ int s_bad;
-  const Shape &sh = pp.sh;
-  const SelectArgs &a = pp.a;
-  sm100::grid_dep_wait();  // the page scores of select_finalize
-  sm100::grid_dep_launch_dependents();
-  const int s = blockIdx.y, h = blockIdx.x;
-  const size_t sh_idx = (size_t)s * sh.Hkv + h;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, sh.P, a.status, false);
-  const int np = (n + sh.P - 1) / sh.P;
-  const int topk_tokens = a.topk[s];
-  int kp = topk_tokens / sh.P;
-  if (kp > sh.kmax || kp < 0 || topk_tokens % sh.P != 0) {
-    if (tid == 0) raise_status(a.status, kStatusBadIndex);
-    kp = max(0, min(kp, sh.kmax));
-  }
-  const float *sc = a.scores + sh_idx * sh.max_pages;
-  int32_t *out = a.idx_out + sh_idx * sh.kmax;
-  const int take = min(kp, np);
-  const bool staged = np <= kTopkSmemKeys;
-  if (tid == 0) s_bad = 0;
-  __syncthreads();
-  int bad = 0;
-  for (int i = tid; i < np; i += kTopkThreads) {
-    const float v = sc[i];
-    bad |= !isfinite(v);
-    if (staged) keys[i] = score_key(v);
-  }
-  if (bad) s_bad = 1;
-  __syncthreads();
-  if (s_bad && tid == 0) raise_status(a.status, kStatusNonfinite);
-  auto key_at = [&](int i) -> uint32_t { return staged ? keys[i] : score_key(sc[i]); };
-
-  if (take >= np) {  // the budget covers the prefix: every page
-    for (int i = tid; i < sh.kmax; i += kTopkThreads) out[i] = i < np ? i : -1;
-    if (tid == 0) a.cnt_out[sh_idx] = np;
-    return;
-  }
+// Threshold key T and the number of keys == T to keep, for 0 < take < n.  Every
+// thread of the CTA calls it.
+template <class KeyAt>
+__device__ __forceinline__ void radix_threshold(int n, int take, KeyAt key_at, TopkScratch &sc,
+                                                uint32_t &thr, uint32_t &need_eq) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = (int)blockDim.x;
   uint32_t prefix = 0, mask = 0;
-  if (tid == 0) s_remaining = (uint32_t)take;
+  if (tid == 0) sc.remaining = (uint32_t)take;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    if (tid < 256) hist[tid] = 0;
+    for (int i = tid; i < 256; i += nt) sc.hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < np; i += kTopkThreads) {
+    for (int i = tid; i < n; i += nt) {
       const uint32_t key = key_at(i);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      if ((key & mask) == prefix) atomicAdd(&sc.hist[(key >> shift) & 255u], 1u);
     }
     __syncthreads();
     if (warp == 0) {
       // lane L owns bins 255-8L down to 248-8L; counts above a lane's bins are
       // the exclusive prefix over the lanes before it
-      const uint32_t rem = s_remaining;
+      const uint32_t rem = sc.remaining;
       uint32_t cnt[8], local = 0;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        cnt[q] = hist[255 - 8 * lane - q];
+        cnt[q] = sc.hist[255 - 8 * lane - q];
         local += cnt[q];
       }
       uint32_t incl = local;
@@ -591,8 +393,8 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk(const __grid_constan
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           if (cum + cnt[q] >= rem) {
-            s_digit = (uint32_t)(255 - 8 * lane - q);
-            s_remaining = rem - cum;
+            sc.digit = (uint32_t)(255 - 8 * lane - q);
+            sc.remaining = rem - cum;
             break;
           }
           cum += cnt[q];
@@ -600,15 +402,25 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk(const __grid_constan
       }
     }
     __syncthreads();
-    prefix |= s_digit << shift;
+    prefix |= sc.digit << shift;
     mask |= 255u << shift;
   }
-  const uint32_t thr = prefix;           // the take-th largest key
-  const uint32_t need_eq = s_remaining;  // keys equal to thr to keep, lowest pages first
+  thr = prefix;
+  need_eq = sc.remaining;
+  __syncthreads();  // sc is reused by the caller
+}
 
-  // ordered compaction: a contiguous chunk per thread, block-wide exclusive scans
-  const int chunk = (np + kTopkThreads - 1) / kTopkThreads;
-  const int i0 = min(np, tid * chunk), i1 = min(np, i0 + chunk);
+// Emits (position, output slot) of the kept keys in ascending position: a
+// contiguous chunk of positions per thread, block-wide exclusive scans of the
+// counts of keys > T and == T; the slot of a kept key is
+// (greater before) + min(equal before, need_eq).
+template <class KeyAt, class Emit>
+__device__ __forceinline__ void ordered_emit(int n, uint32_t thr, uint32_t need_eq, KeyAt key_at,
+                                             Emit emit, TopkScratch &sc) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = (int)blockDim.x;
+  const int warps = nt >> 5;
+  const int chunk = (n + nt - 1) / nt;
+  const int i0 = min(n, tid * chunk), i1 = min(n, i0 + chunk);
   uint32_t n_eq = 0, n_gt = 0;
   for (int i = i0; i < i1; ++i) {
     const uint32_t key = key_at(i);
@@ -625,12 +437,12 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk(const __grid_constan
     }
   }
   if (lane == 31) {
-    scan_eq[warp] = e;
-    scan_gt[warp] = g;
+    sc.scan_eq[warp] = e;
+    sc.scan_gt[warp] = g;
   }
   __syncthreads();
   if (warp == 0) {
-    uint32_t we = scan_eq[lane], wg = scan_gt[lane];
+    uint32_t we = lane < warps ? sc.scan_eq[lane] : 0u, wg = lane < warps ? sc.scan_gt[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t e2 = __shfl_up_sync(0xffffffffu, we, o), g2 = __shfl_up_sync(0xffffffffu, wg, o);
@@ -639,31 +451,670 @@ __global__ void __launch_bounds__(kTopkThreads) select_topk(const __grid_constan
         wg += g2;
       }
     }
-    scan_eq[lane] = we;
-    scan_gt[lane] = wg;
+    sc.scan_eq[lane] = we;
+    sc.scan_gt[lane] = wg;
   }
   __syncthreads();
-  uint32_t eq_before = e - n_eq + (warp > 0 ? scan_eq[warp - 1] : 0u);
-  uint32_t gt_before = g - n_gt + (warp > 0 ? scan_gt[warp - 1] : 0u);
-  // position of a kept page = kept pages before it = (greater before) + min(equal before, need_eq)
+  uint32_t eq_before = e - n_eq + (warp > 0 ? sc.scan_eq[warp - 1] : 0u);
+  uint32_t gt_before = g - n_gt + (warp > 0 ? sc.scan_gt[warp - 1] : 0u);
   for (int i = i0; i < i1; ++i) {
     const uint32_t key = key_at(i);
     if (key > thr) {
-      out[gt_before + min(eq_before, need_eq)] = i;
+      emit(i, (int)(gt_before + min(eq_before, need_eq)));
       ++gt_before;
     } else if (key == thr) {
-      if (eq_before < need_eq) out[gt_before + eq_before] = i;
+      if (eq_before < need_eq) emit(i, (int)(gt_before + eq_before));
       ++eq_before;
     }
   }
-  for (int i = take + tid; i < sh.kmax; i += kTopkThreads) out[i] = -1;
-  if (tid == 0) a.cnt_out[sh_idx] = take;
+  __syncthreads();  // sc is reused by the caller
+}
+
+// The take largest of n keys (ties to the lower position), emitted in ascending
+// position; every key when take >= n.
+template <class KeyAt, class Emit>
+__device__ __forceinline__ void block_topk(int n, int take, KeyAt key_at, Emit emit, TopkScratch &sc) {
+  if (take <= 0 || n <= 0) return;
+  if (take >= n) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) emit(i, i);
+    return;
+  }
+  uint32_t thr, need_eq;
+  radix_threshold(n, take, key_at, sc, thr, need_eq);
+  ordered_emit(n, thr, need_eq, key_at, emit, sc);
+}
+
+// ---------------------------------------------------------------------------
+// Warp-level top-k for kp <= 128 (the fast path).  A candidate is a 64-bit key
+// (score bits << 32) | ~page: keys order by score, then by lower page, and are
+// all distinct; 0 pads (below every real key).  A warp holds a list of
+// P = 32 E keys, key i = lane + 32 j in register j, and sorts or merges it with
+// bitonic networks of shuffles.
+// ---------------------------------------------------------------------------
+constexpr int kFastTopk = 128;  // largest kp of the fast path
+
+__device__ __forceinline__ uint64_t cand_key(float score, int page) {
+  return ((uint64_t)score_key(score) << 32) | (uint32_t)~(uint32_t)page;
+}
+__device__ __forceinline__ int cand_page(uint64_t key) { return (int)~(uint32_t)key; }
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// One compare-exchange stage (distance d) of a bitonic network over the warp's
+// list, in sub-sequences of length k: a pair (i, i + d) ends larger-first where
+// (i & k) == 0 and smaller-first elsewhere.
+template <int E>
+__device__ __forceinline__ void bitonic_stage(uint64_t (&x)[E], int k, int d, int lane) {
+  if (d >= 32) {
+    const int dj = d >> 5;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      if (j & dj) continue;
+      const int jp = j | dj;
+      const bool desc = ((lane + 32 * j) & k) == 0;
+      const uint64_t a = x[j], b = x[jp];
+      const bool swap = desc ? (a < b) : (a > b);
+      x[j] = swap ? b : a;
+      x[jp] = swap ? a : b;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      const int i = lane + 32 * j;
+      const uint64_t y = shfl_xor_u64(x[j], d);
+      const bool keep_max = ((i & d) == 0) == ((i & k) == 0);
+      x[j] = keep_max ? (x[j] > y ? x[j] : y) : (x[j] < y ? x[j] : y);
+    }
+  }
+}
+
+// Sorts the warp's list in descending order.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(uint64_t (&x)[E], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32 * E; k <<= 1)
+#pragma unroll
+    for (int d = k >> 1; d > 0; d >>= 1) bitonic_stage<E>(x, k, d, lane);
+}
+
+// x, y sorted descending: x becomes the P largest of x and y, sorted descending
+// (max(x_i, y_{P-1-i}) is a bitonic sequence holding them; a bitonic merge sorts it).
+template <int E>
+__device__ __forceinline__ void warp_merge_top(uint64_t (&x)[E], const uint64_t (&y)[E], int lane) {
+#pragma unroll
+  for (int j = 0; j < E; ++j) {
+    const uint64_t r = shfl_u64(y[E - 1 - j], 31 - lane);
+    x[j] = x[j] > r ? x[j] : r;
+  }
+#pragma unroll
+  for (int d = 16 * E; d > 0; d >>= 1) bitonic_stage<E>(x, 64 * E, d, lane);
+}
+
+// Every warp holds a sorted list; afterwards warp 0 holds the P largest of all
+// of them, sorted descending.  wl: shared memory for (warps) lists.  Every
+// thread of the CTA calls it.
+template <int E>
+__device__ __forceinline__ void block_merge_lists(uint64_t (&x)[E], uint64_t *wl) {
+  constexpr int P = 32 * E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, warps = (int)blockDim.x >> 5;
+#pragma unroll
+  for (int j = 0; j < E; ++j) wl[warp * P + lane + 32 * j] = x[j];
+  __syncthreads();
+  for (int st = 1; st < warps; st <<= 1) {
+    if (warp % (2 * st) == 0 && warp + st < warps) {
+      uint64_t y[E];
+#pragma unroll
+      for (int j = 0; j < E; ++j) y[j] = wl[(warp + st) * P + lane + 32 * j];
+      warp_merge_top<E>(x, y, lane);
+#pragma unroll
+      for (int j = 0; j < E; ++j) wl[warp * P + lane + 32 * j] = x[j];
+    }
+    __syncthreads();
+  }
+}
+
+// Final selection (fast path), one CTA: the take largest keys over the G
+// candidate lists (each P keys, sorted descending, in global memory), written
+// to out[0..take) as ascending pages, out[take..kmax) = -1.
+template <int E>
+__device__ __forceinline__ void final_topk_fast(const uint64_t *lists, size_t list_stride, int G, int take,
+                                                int32_t *out, int kmax, uint64_t *wl) {
+  constexpr int P = 32 * E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, warps = (int)blockDim.x >> 5;
+  uint64_t x[E];
+#pragma unroll
+  for (int j = 0; j < E; ++j) x[j] = 0;
+  // one list ahead in flight
+  uint64_t nx[E];
+  if (warp < G) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) nx[j] = __ldcg(lists + (size_t)warp * list_stride + lane + 32 * j);
+  }
+  for (int c = warp; c < G; c += warps) {
+    uint64_t y[E];
+#pragma unroll
+    for (int j = 0; j < E; ++j) y[j] = nx[j];
+    if (c + warps < G) {
+#pragma unroll
+      for (int j = 0; j < E; ++j) nx[j] = __ldcg(lists + (size_t)(c + warps) * list_stride + lane + 32 * j);
+    }
+    if (c == warp) {
+#pragma unroll
+      for (int j = 0; j < E; ++j) x[j] = y[j];
+    } else {
+      warp_merge_top<E>(x, y, lane);
+    }
+  }
+  block_merge_lists<E>(x, wl);
+  if (warp == 0) {
+    // the take largest, re-sorted by ascending page: descending order of ~page
+#pragma unroll
+    for (int j = 0; j < E; ++j) x[j] = (lane + 32 * j < take) ? (x[j] & 0xffffffffull) : 0ull;
+    warp_sort_desc<E>(x, lane);
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      const int i = lane + 32 * j;
+      if (i < kmax) out[i] = i < take ? cand_page(x[j]) : -1;
+    }
+  }
+  for (int i = P + (int)threadIdx.x; i < kmax; i += blockDim.x) out[i] = -1;
+}
+
+// Candidate list of one warp, built while the warp scores its tiles (fast path,
+// E > 0): x holds the warp's P = 32 E largest keys so far, sorted descending;
+// keys of newly scored pages collect in the warp's pend[0..P) and are sorted
+// and merged into x whenever P of them are pending.
+template <int E>
+struct WarpCands {
+  uint64_t x[E > 0 ? E : 1];
+  uint64_t *pend;
+  int npend;  // warp-uniform
+  __device__ __forceinline__ void init(uint64_t *p) {
+#pragma unroll
+    for (int j = 0; j < (E > 0 ? E : 1); ++j) x[j] = 0;
+    pend = p;
+    npend = 0;
+  }
+  __device__ __forceinline__ void flush(int lane) {
+    if constexpr (E > 0) {
+      __syncwarp();
+      uint64_t y[E];
+#pragma unroll
+      for (int j = 0; j < E; ++j) y[j] = lane + 32 * j < npend ? pend[lane + 32 * j] : 0ull;
+      __syncwarp();
+      warp_sort_desc<E>(y, lane);
+      warp_merge_top<E>(x, y, lane);
+      npend = 0;
+    }
+  }
+};
+
+// Stage-and-score loop of one CTA: tiles [tl0, tl1) of its (sequence, KV head),
+// in batches of cap_t tiles through kStageBufs shared buffers (bulk copies of
+// the tile maxima and unit masses; while one batch is scored the next
+// kStageBufs - 1 are in flight).  start() issues the first kStageBufs batches;
+// thread 0 issues each later one as its buffer is freed.
+constexpr int kStageBufs = 4;
+struct ScoreStager {
+  const float *mt_head, *pp_head;  // [max_tiles][BGp], [max_tiles][BGp][units] of the head
+  unsigned char *buf0;             // shared buffers, buf_bytes apart
+  uint32_t bar0;                   // their mbarriers, 8 bytes apart (shared addresses)
+  int tl0, tl1, cap_t, BGp, units, buf_bytes;
+
+  __device__ __forceinline__ int batches() const { return tl1 > tl0 ? (tl1 - tl0 + cap_t - 1) / cap_t : 0; }
+  __device__ __forceinline__ unsigned char *buf(int b) const { return buf0 + (size_t)(b % kStageBufs) * buf_bytes; }
+  __device__ __forceinline__ uint32_t bar(int b) const { return bar0 + 8u * (uint32_t)(b % kStageBufs); }
+  __device__ __forceinline__ uint32_t parity(int b) const { return (uint32_t)((b / kStageBufs) & 1); }
+  __device__ __forceinline__ const float *mt_buf(int b) const { return reinterpret_cast<const float *>(buf(b)); }
+  __device__ __forceinline__ const float *pp_buf(int b) const {
+    return reinterpret_cast<const float *>(buf(b) + (size_t)cap_t * BGp * 4);
+  }
+  // thread 0 only
+  __device__ __forceinline__ void issue(int b) const {
+    const int t0 = tl0 + b * cap_t, nt = min(cap_t, tl1 - t0);
+    const uint32_t mt_bytes = (uint32_t)nt * BGp * 4, pp_bytes = mt_bytes * units;
+    sm100::mbar_arrive_expect_tx(bar(b), mt_bytes + pp_bytes);
+    sm100::bulk_load(smem_addr(buf(b)), mt_head + (size_t)t0 * BGp, mt_bytes, bar(b));
+    sm100::bulk_load(smem_addr(buf(b) + (size_t)cap_t * BGp * 4), pp_head + (size_t)t0 * BGp * units, pp_bytes,
+                     bar(b));
+  }
+  // thread 0 only: barrier set-up and the first batches
+  __device__ __forceinline__ void start() const {
+#pragma unroll
+    for (int i = 0; i < kStageBufs; ++i) sm100::mbar_init(bar0 + 8u * i, 1);
+    sm100::fence_mbar_init();
+    const int nb = batches();
+    for (int b = 0; b < kStageBufs && b < nb; ++b) issue(b);
+  }
+};
+
+// Page scores of nt tiles staged in shared memory, tile t being tile0 + t of the
+// (sequence, KV head): mt [nt][BGp] tile maxima, pp [nt][BGp][units] unit
+// masses.  One warp per tile; lane l takes the rows l + 32 c < BG, whose M and
+// 1/L (rm, rl) it holds in registers.  Scores of pages below p_hi go to
+// gout[page] and sout[page - p_lo] and, with E > 0, into the warp's candidates;
+// a non-finite score (a non-finite input row) is reported in the status word.
+template <int PAGE, int kRowChunks, int E>
+__device__ __forceinline__ void scores_from_smem(const float *mt, const float *pp, int nt, int tile0,
+                                                 int BG, int BGp, const float (&rm)[kRowChunks],
+                                                 const float (&rl)[kRowChunks], float inv_bg, int p_lo,
+                                                 int p_hi, float *gout, float *sout, uint32_t *status,
+                                                 WarpCands<E> &wc) {
+  using U = tc::Units<PAGE>;
+  constexpr int kUnits = U::kPerTile;
+  constexpr int kPagesPerTile = tc::kBN / PAGE;
+  using W = typename std::conditional<kUnits == 4, float4, float2>::type;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, warps = (int)blockDim.x >> 5;
+  constexpr int kT = 2;  // tiles a warp scores at once (independent chains)
+  for (int t0 = warp; t0 < nt; t0 += kT * warps) {
+    float acc[kT][kUnits];
+#pragma unroll
+    for (int tt = 0; tt < kT; ++tt)
+#pragma unroll
+      for (int u = 0; u < kUnits; ++u) acc[tt][u] = 0.f;
+#pragma unroll
+    for (int c = 0; c < kRowChunks; ++c) {
+      const int row = lane + 32 * c;
+      if (row < BG) {  // (rows past BG hold no data; a non-finite row makes the scores non-finite)
+#pragma unroll
+        for (int tt = 0; tt < kT; ++tt) {
+          const int t = t0 + tt * warps;
+          if (t < nt) {
+            const float f = exp2f(mt[t * BGp + row] - rm[c]) * rl[c];
+            const W w = reinterpret_cast<const W *>(pp)[t * BGp + row];
+            const float *wu = reinterpret_cast<const float *>(&w);
+#pragma unroll
+            for (int u = 0; u < kUnits; ++u) acc[tt][u] = fmaf(wu[u], f, acc[tt][u]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < kT; ++tt) {
+      const int t = t0 + tt * warps;
+      if (t >= nt) break;  // (warp-uniform)
+      float pv[kPagesPerTile];
+#pragma unroll
+      for (int pi = 0; pi < kPagesPerTile; ++pi) {
+        pv[pi] = 0.f;
+#pragma unroll
+        for (int u = pi * U::kPerPage; u < (pi + 1) * U::kPerPage; ++u) pv[pi] += acc[tt][u];
+      }
+      const float v = warp_sum_multi<kPagesPerTile>(pv, lane) * inv_bg;
+      const int pi = lane / (32 / kPagesPerTile);
+      const int page = (tile0 + t) * kPagesPerTile + pi;
+      const bool owner = lane % (32 / kPagesPerTile) == 0, live = page < p_hi;
+      if (owner && live) {
+        gout[page] = v;
+        if (sout) sout[page - p_lo] = v;
+        if (!isfinite(v)) raise_status(status, kStatusNonfinite);
+      }
+      if constexpr (E > 0) {
+        if (owner) wc.pend[wc.npend + pi] = live ? cand_key(v, page) : 0ull;
+        wc.npend += kPagesPerTile;
+        if (wc.npend == 32 * E) wc.flush(lane);
+      }
+    }
+  }
+}
+
+// Scores every staged batch of a ScoreStager (all threads of the CTA); with
+// E > 0 each warp also builds its candidate list and the CTA's P largest keys
+// end in `slot` (sorted descending, 0-padded), through the warp lists in wl.
+template <int PAGE, int kRC, int E>
+__device__ __forceinline__ void score_batches(const ScoreStager &st, const float *sM, const float *sLinv,
+                                              int BG, float inv_bg, int p_lo, int p_hi, float *gout,
+                                              float *sout, uint32_t *status, const sm100::WaitCtx &ctx,
+                                              uint64_t *wl, uint64_t *slot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float rm[kRC], rl[kRC];
+#pragma unroll
+  for (int c = 0; c < kRC; ++c) {
+    const int row = lane + 32 * c;
+    rm[c] = row < BG ? sM[row] : 0.f;
+    rl[c] = row < BG ? sLinv[row] : 0.f;
+  }
+  WarpCands<E> wc;
+  wc.init(wl + (size_t)warp * 32 * (E > 0 ? E : 1));
+  const int nb = st.batches();
+  for (int b = 0; b < nb; ++b) {
+    sm100::mbar_wait(st.bar(b), st.parity(b), ctx);
+    const int t0 = st.tl0 + b * st.cap_t;
+    scores_from_smem<PAGE, kRC, E>(st.mt_buf(b), st.pp_buf(b), min(st.cap_t, st.tl1 - t0), t0, BG, st.BGp,
+                                   rm, rl, inv_bg, p_lo, p_hi, gout, sout, status, wc);
+    __syncthreads();  // every read of this buffer is done before it is refilled
+    if (threadIdx.x == 0 && b + kStageBufs < nb) {
+      sm100::fence_proxy_async_smem();
+      st.issue(b + kStageBufs);
+    }
+  }
+  if constexpr (E > 0) {
+    if (wc.npend > 0) wc.flush(lane);
+  }
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(39);
+  if constexpr (E > 0) {
+    block_merge_lists<E>(wc.x, wl);
+    if (warp == 0) {
+#pragma unroll
+      for (int j = 0; j < E; ++j) slot[lane + 32 * j] = wc.x[j];
+    }
+  }
+  __syncthreads();
+}
+
+// Shared memory of the tail (steps 2-4): the engine's whole layout is free once
+// it has been torn down.  [0, 1K) sM, [1K, 2K) sLinv, [2K, ..) TopkScratch,
+// kOffTailBars: the staging buffers' mbarriers; kTailHead: the warps' candidate
+// lists (fast path); kOffSf: the CTA's page scores, then the staging buffers.
+constexpr int kOffTailBars = 3584;
+// A CTA that arrives at the group barrier with more than this many CTAs of the
+// group still to come starts its staging copies before it waits.
+constexpr int kPrefetchMargin = 3;
+constexpr int kTailHead = 4096;
+constexpr int kOffSf = kTailHead + (tc::kThreads / 32) * kFastTopk * 8;
+template <int D>
+constexpr int tail_bytes() { return (int)tc::Layout<D, kSelStages>::kOffBar; }
+// the page scores take at most a quarter of what follows kOffSf; the rest holds
+// the staging buffers, each at least one tile
+static_assert((tail_bytes<64>() - kOffSf) * 3 / 4 / 4 >= 256 * 4 * 5, "staging buffer");
+
+template <int D, int PAGE>
+__global__ void __launch_bounds__(tc::kThreads, 1)
+    select_fused(const __grid_constant__ PartialParams pp, const __grid_constant__ CUtensorMap kmap,
+                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kmap4,
+                 const __grid_constant__ CUtensorMap vmap4) {
+  extern __shared__ unsigned char smem_raw[];
+  const Shape &sh = pp.sh;
+  const SelectPlan &plan = pp.plan;
+  const SelectArgs &a = pp.a;
+  const int G = plan.group_ctas;
+  const int gl = blockIdx.x / G, c = blockIdx.x % G;  // group of this launch, CTA in the group
+  const int group = pp.group0 + gl;
+  const int s = group / sh.Hkv, h = group % sh.Hkv;
+  const int split = c / plan.rowtiles, rt = c % plan.rowtiles;
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
+  SelectPolicy<D, PAGE> pol;
+  pol.kmap = &kmap;
+  pol.vmap = &vmap;
+  pol.kmap4 = &kmap4;
+  pol.vmap4 = &vmap4;
+  tc::Engine<D, kSelStages> eng;
+  eng.setup(smem_raw, pol);
+  // everything below may read what the kernel ahead of this one wrote
+  sm100::grid_dep_wait();
+  sm100::grid_dep_launch_dependents();
+
+  // ---- 1. split-KV attention ----
+  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, PAGE, a.status, threadIdx.x == 0 && c == 0);
+  const int ntiles = (n + tc::kBN - 1) / tc::kBN;
+  const int t_begin = split * plan.tiles_per_split;
+  const int num_tiles = max(0, min(ntiles, t_begin + plan.tiles_per_split) - t_begin);
+  const size_t sh_idx = (size_t)s * sh.Hkv + h;
+  pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
+  pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
+  pol.mtile_head = a.mtile + sh_idx * plan.max_tiles * plan.bgp;
+  pol.pagepart_head = a.pagepart + sh_idx * plan.max_tiles * plan.bgp * tc::Units<PAGE>::kPerTile;
+  pol.status = a.status;
+  pol.n_phys = sh.n_phys;
+  pol.phys0 = (long long)s * sh.max_pages;
+  pol.Hkv = sh.Hkv;
+  pol.h = h;
+  pol.G = sh.G;
+  pol.Hq = sh.Hq;
+  pol.BG = sh.BG;
+  pol.BGp = plan.bgp;
+  pol.n = n;
+  pol.np = (n + PAGE - 1) / PAGE;
+  pol.t_begin = t_begin;
+  pol.row_base = rt * kRowsPerCta;
+  pol.report = rt == 0;
+  pol.sl2 = sh.sl2;
+  eng.init(a.status, pol, num_tiles);
+  float m, l;
+  eng.template run<PAGE>(pol, num_tiles, m, l);
+  float m_row, l_row, wa, wb;
+  eng.finish(m, l, m_row, l_row, wa, wb);
+  if (eng.warp >= 2) {
+    // O = wa * O_0 + wb * O_1 relative to m_row; this thread writes its half of the columns
+    const int g = eng.group();
+    const int row = rt * kRowsPerCta + eng.row_in_tile();
+    const bool row_ok = row < sh.BG;
+    const size_t prow = ((sh_idx * plan.splits + split) * sh.BG + row);
+#pragma unroll
+    for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 32) {
+      uint32_t oa[32], ob[32];
+      eng.load_o(0, c0, oa);
+      eng.load_o(1, c0, ob);
+      if (row_ok && l_row > 0.f) {
+        float4 *dst = reinterpret_cast<float4 *>(a.part_o + prow * D + c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = wa > 0.f ? wa * __uint_as_float(oa[4 * i + e]) : 0.f;
+            const float x1 = wb > 0.f ? wb * __uint_as_float(ob[4 * i + e]) : 0.f;
+            v[e] = x0 + x1;
+          }
+#if DSA_PART_EVICT_LAST
+          sm100::st_hint(dst + i, make_float4(v[0], v[1], v[2], v[3]), sm100::l2_policy_evict_last());
+#else
+          dst[i] = make_float4(v[0], v[1], v[2], v[3]);
+#endif
+        }
+      }
+    }
+    if (row_ok && g == 0)
+      *reinterpret_cast<float2 *>(a.part_ml + prow * 2) =
+          l_row > 0.f ? make_float2(m_row, l_row) : make_float2(-INFINITY, 0.f);
+    if (row == rt * kRowsPerCta) DSA_TRACE_EVENT(7);
+  }
+  eng.teardown();  // ends with a __syncthreads: every partial of this CTA is written
+
+  // ---- staging of this CTA's page partials (tile maxima, unit masses) ----
+  constexpr int kPagesPerTile = tc::kBN / PAGE;
+  constexpr int kUnits = tc::Units<PAGE>::kPerTile;
+  unsigned char *tail = eng.smem;
+  float *sM = reinterpret_cast<float *>(tail);
+  float *sLinv = sM + 256;
+  TopkScratch &sc = *reinterpret_cast<TopkScratch *>(tail + 2048);
+  static_assert(2048 + sizeof(TopkScratch) <= kOffTailBars, "tail header");
+  const int np = (n + PAGE - 1) / PAGE;
+  const int per_rt = (num_tiles + plan.rowtiles - 1) / plan.rowtiles;
+  const int tl0 = t_begin + min(num_tiles, rt * per_rt);
+  const int tl1 = t_begin + min(num_tiles, (rt + 1) * per_rt);
+  const int p0 = tl0 * kPagesPerTile;
+  const int p1 = max(p0, min(np, tl1 * kPagesPerTile));
+  const int n_loc = p1 - p0;
+  const int BGp = plan.bgp;
+  const bool aborted = *eng.abort_flag() != 0;
+  uint64_t *wl = reinterpret_cast<uint64_t *>(tail + kTailHead);
+  const int sf_bytes = (n_loc * 4 + 15) & ~15;
+  const bool staged = sf_bytes <= (tail_bytes<D>() - kOffSf) / 4;
+  float *sf = reinterpret_cast<float *>(tail + kOffSf);
+  const int off_buf = kOffSf + (staged ? sf_bytes : 0);
+  const int tile_bytes = BGp * 4 * (1 + kUnits);
+  ScoreStager st;
+  st.mt_head = a.mtile + sh_idx * plan.max_tiles * BGp;
+  st.pp_head = a.pagepart + sh_idx * plan.max_tiles * BGp * kUnits;
+  st.cap_t = (tail_bytes<D>() - off_buf) / (kStageBufs * tile_bytes);  // >= 1 (see kOffSf)
+  st.buf_bytes = st.cap_t * tile_bytes;
+  st.buf0 = tail + off_buf;
+  st.bar0 = smem_addr(tail + kOffTailBars);
+  st.tl0 = tl0;
+  st.tl1 = aborted ? tl0 : tl1;  // nothing is staged after an abort
+  st.BGp = BGp;
+  st.units = kUnits;
+  // With one row tile the CTA scores only tiles it wrote itself.  A CTA that
+  // will wait at the group barrier (several CTAs of the group still to come)
+  // starts their copies before waiting; the late ones load the row statistics
+  // first, so that those loads are not queued behind the copies.
+  const bool own_rows = plan.rowtiles == 1;
+  sm100::fence_proxy_async_global();  // this thread's partial stores, before any bulk copy
+  __syncthreads();
+
+  // ---- 2. group barrier ----
+  uint32_t *arrive = a.counters + 4 * gl, *leave = arrive + 1, *orows = arrive + 2, *odone = arrive + 3;
+  const int topk_tokens = a.topk[s];  // (in flight during the wait)
+  if (threadIdx.x == 0) {
+    DSA_TRACE_EVENT(40);
+    const uint32_t prev = sm100::arrive_gpu(arrive);
+    sc.flag = own_rows && (int)prev + kPrefetchMargin < G;
+  }
+  __syncthreads();
+  const bool started = sc.flag;
+  if (started && threadIdx.x == 0) st.start();
+  if (threadIdx.x == 0) {
+    if (!sm100::wait_count_geq(arrive, (uint32_t)G)) sm100::note_timeout(a.status, 0xffu);
+    DSA_TRACE_EVENT(41);
+  }
+  sm100::fence_proxy_async_global();  // the other CTAs' partials, before the bulk copies
+  __syncthreads();
+
+  // ---- 3. row statistics, page scores, local candidates ----
+  int kp = topk_tokens / PAGE;
+  if (kp > sh.kmax || kp < 0 || topk_tokens % PAGE != 0) {
+    if (threadIdx.x == 0 && c == 0) raise_status(a.status, kStatusBadIndex);
+    kp = max(0, min(kp, sh.kmax));
+  }
+  const int take = min(kp, np);
+  const bool every_page = take >= np;
+  const bool fast = kp <= kFastTopk;
+  const int E = every_page ? 0 : (!fast ? 0 : (kp <= 32 ? 1 : (kp <= 64 ? 2 : 4)));
+  merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv, [&]() {
+    if (threadIdx.x == 0 && !started) st.start();
+  });
+  __syncthreads();
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(31);
+  float *gs = a.scores + sh_idx * sh.max_pages;
+  const size_t cslot = sh_idx * G + c;
+  uint64_t *slot = a.cand + cslot * plan.slot_len;
+  {
+    const float inv_bg = 1.f / (float)sh.BG;
+    float *sout = staged ? sf : nullptr;
+#define DSA_SCORE(KRC, EE)                                                                                   \
+  score_batches<PAGE, KRC, EE>(st, sM, sLinv, sh.BG, inv_bg, p0, p1, gs, sout, a.status, eng.ctx, wl, slot)
+    if (BGp <= 128) {
+      if (E == 0) DSA_SCORE(4, 0); else if (E == 1) DSA_SCORE(4, 1); else if (E == 2) DSA_SCORE(4, 2); else DSA_SCORE(4, 4);
+    } else {
+      if (E == 0) DSA_SCORE(8, 0); else if (E == 1) DSA_SCORE(8, 1); else if (E == 2) DSA_SCORE(8, 2); else DSA_SCORE(8, 4);
+    }
+#undef DSA_SCORE
+  }
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(44);
+  // (score_batches ends with a __syncthreads: sf, the slot and this CTA's part of
+  // a.scores are complete)
+  if (!every_page && !fast) {
+    const int take_loc = min(take, n_loc);
+    auto score_at = [&](int i) -> float { return staged ? sf[i] : __ldcg(gs + p0 + i); };
+    auto key_loc = [&](int i) -> uint32_t { return score_key(score_at(i)); };
+    block_topk(n_loc, take_loc, key_loc, [&](int i, int pos) { slot[pos] = cand_key(score_at(i), p0 + i); },
+               sc);
+    if (threadIdx.x == 0) a.ccnt[cslot] = take_loc;
+  }
+  if (threadIdx.x == 0) DSA_TRACE_EVENT(46);
+
+  // ---- 4. the group's last CTA selects among the candidates; every CTA then
+  //      merges output rows, taken from a counter ----
+  __syncthreads();  // every candidate of this CTA is written
+  if (threadIdx.x == 0) {
+    DSA_TRACE_EVENT(42);
+    const uint32_t prev = sm100::arrive_gpu(leave);
+    sc.flag = prev == (uint32_t)G - 1u;
+    if (sc.flag) __threadfence();  // the other CTAs' candidates are visible from here on
+  }
+  __syncthreads();
+  if (sc.flag) {
+    int32_t *out = a.idx_out + sh_idx * sh.kmax;
+    const uint64_t *lists = a.cand + sh_idx * G * plan.slot_len;
+    if (every_page) {
+      for (int i = threadIdx.x; i < sh.kmax; i += blockDim.x) out[i] = i < np ? i : -1;
+    } else if (fast) {
+      if (E == 1) final_topk_fast<1>(lists, plan.slot_len, G, take, out, sh.kmax, wl);
+      else if (E == 2) final_topk_fast<2>(lists, plan.slot_len, G, take, out, sh.kmax, wl);
+      else final_topk_fast<4>(lists, plan.slot_len, G, take, out, sh.kmax, wl);
+    } else {
+      // offsets of the CTAs' candidate lists (CTA order is page order)
+      int *offs = reinterpret_cast<int *>(tail + kTailHead);
+      const int offs_bytes = ((G + 1) * 4 + 15) & ~15;
+      uint64_t *cs = reinterpret_cast<uint64_t *>(tail + kTailHead + offs_bytes);
+      const int cap = (tail_bytes<D>() - kTailHead - offs_bytes) / 8;
+      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, warps = (int)blockDim.x >> 5;
+      if (warp == 0) {
+        int carry = 0;
+        for (int j0 = 0; j0 < G; j0 += 32) {
+          const int v = j0 + lane < G ? min(max(__ldcg(a.ccnt + sh_idx * G + j0 + lane), 0), sh.kmax) : 0;
+          int incl = v;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+          }
+          if (j0 + lane < G) offs[j0 + lane] = carry + incl - v;
+          carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) offs[G] = carry;
+      }
+      __syncthreads();
+      const int ncand = offs[G];
+      if (ncand <= cap) {
+        for (int j = warp; j < G; j += warps) {
+          const uint64_t *src = lists + (size_t)j * plan.slot_len;
+          const int o = offs[j], cnt = offs[j + 1] - o;
+          for (int i = lane; i < cnt; i += 32) cs[o + i] = __ldcg(src + i);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) DSA_TRACE_EVENT(47);
+        block_topk(ncand, take, [&](int i) -> uint32_t { return (uint32_t)(cs[i] >> 32); },
+                   [&](int i, int pos) { out[pos] = cand_page(cs[i]); }, sc);
+      } else {  // too many candidates to stage: select over every page score of the head
+        block_topk(np, take, [&](int i) -> uint32_t { return score_key(__ldcg(gs + i)); },
+                   [&](int i, int pos) { out[pos] = i; }, sc);
+      }
+      for (int i = take + threadIdx.x; i < sh.kmax; i += blockDim.x) out[i] = -1;
+    }
+    if (threadIdx.x == 0) {
+      a.cnt_out[sh_idx] = take;
+      DSA_TRACE_EVENT(43);
+    }
+  }
+  {
+    const int warp = threadIdx.x >> 5, warps = (int)blockDim.x >> 5;
+    for (;;) {
+      __syncthreads();  // the previous row block is taken
+      if (threadIdx.x == 0) sc.digit = atomicAdd(orows, (uint32_t)warps);
+      __syncthreads();
+      const int base = (int)sc.digit;
+      if (base >= sh.BG) break;
+      if (base + warp < sh.BG) merge_output_row<D>(sh, plan, a, sh_idx, s, h, base + warp, sM, sLinv);
+    }
+  }
+  if (threadIdx.x == 0) {
+    // the group's last CTA to find no rows left resets the counters: every CTA
+    // of the group has passed them all
+    if (atomicAdd(odone, 1u) == (uint32_t)G - 1u) {
+      *arrive = 0u;
+      *leave = 0u;
+      *orows = 0u;
+      *odone = 0u;
+    }
+    DSA_TRACE_EVENT(45);
+  }
 }
 
 template <int D, int PAGE>
 cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectArgs &a,
                          cudaStream_t stream) {
-  PartialParams pp{sh, plan, a};
+  PartialParams pp{sh, plan, a, 0};
   CUtensorMap kmap, vmap;
   const long long rows = sh.n_phys * sh.Hkv * PAGE;
   cudaError_t err = make_kv_tensor_map(&kmap, a.k, rows, D, PAGE);
@@ -675,35 +1126,31 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
   if (err != cudaSuccess) return err;
   err = make_kv_pages_tensor_map(&vmap4, a.v, sh.n_phys, sh.Hkv, PAGE, D, tc::kBN / PAGE);
   if (err != cudaSuccess) return err;
-  constexpr auto kern = select_partial<D, PAGE>;
+  constexpr auto kern = select_fused<D, PAGE>;
   constexpr size_t smem = tc::Layout<D, kSelStages>::kAlloc;
   err = set_smem_once<kern>(smem);
   if (err != cudaSuccess) return err;
-  // all three kernels are programmatic dependents of the kernel ahead of them:
-  // each one's set-up overlaps the tail of the previous one
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  // Cooperative: the CTAs of a launch are co-resident, which the group barrier
+  // needs.  Programmatic dependent: the set-up overlaps the tail of the kernel
+  // ahead on the stream.
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeCooperative;
+  attrs[0].val.cooperative = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.stream = stream;
-  cfg.attrs = pdl;
-  cfg.numAttrs = 1;
-  cfg.gridDim = dim3(plan.splits * plan.rowtiles, sh.Hkv, sh.S);
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
   cfg.blockDim = dim3(tc::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
-  err = cudaLaunchKernelEx(&cfg, kern, pp, kmap, vmap, kmap4, vmap4);
-  if (err != cudaSuccess) return err;
-  const int score_ctas = (sh.max_pages + plan.fin_pages - 1) / plan.fin_pages;
-  const int o_ctas = (sh.BG + kRowsPerFinCta - 1) / kRowsPerFinCta;
-  cfg.gridDim = dim3(score_ctas + o_ctas, sh.Hkv, sh.S);
-  cfg.blockDim = dim3(kFinThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  err = cudaLaunchKernelEx(&cfg, select_finalize<D, PAGE>, pp);
-  if (err != cudaSuccess) return err;
-  cfg.gridDim = dim3(sh.Hkv, sh.S, 1);
-  cfg.blockDim = dim3(kTopkThreads, 1, 1);
-  err = cudaLaunchKernelEx(&cfg, select_topk, pp);
-  if (err != cudaSuccess) return err;
+  const int groups = sh.S * sh.Hkv;
+  for (int g0 = 0; g0 < groups; g0 += plan.groups_per_launch) {
+    pp.group0 = g0;
+    cfg.gridDim = dim3(std::min(plan.groups_per_launch, groups - g0) * plan.group_ctas, 1, 1);
+    err = cudaLaunchKernelEx(&cfg, kern, pp, kmap, vmap, kmap4, vmap4);
+    if (err != cudaSuccess) return err;
+  }
   return cudaGetLastError();
 }
 
@@ -722,23 +1169,33 @@ SelectPlan plan_select(const Shape &sh, int num_sms) {
   splits = std::min(splits, p.max_tiles);
   p.tiles_per_split = (p.max_tiles + splits - 1) / splits;
   p.splits = (p.max_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  // rows of the tile maxima / unit masses padded to 4 (16-byte aligned tile blocks)
+  p.bgp = (sh.BG + 3) & ~3;
+  // candidate list of a CTA: kp <= 128 keeps a power of two >= 32 of them
+  if (sh.kmax <= kFastTopk) {
+    p.slot_len = 32;
+    while (p.slot_len < sh.kmax) p.slot_len *= 2;
+  } else {
+    p.slot_len = sh.kmax;
+  }
+  // groups of one launch: all of their CTAs resident at once
+  p.group_ctas = p.splits * p.rowtiles;
+  p.groups_per_launch = (int)std::max(1LL, std::min<long long>(kMaxGroupsPerLaunch, num_sms / p.group_ctas));
+  const long long groups = (long long)sh.S * sh.Hkv;
+  p.groups_per_launch = (int)std::min<long long>(p.groups_per_launch, groups);
+  p.launches = (int)((groups + p.groups_per_launch - 1) / p.groups_per_launch);
   auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
-  size_t off = 4096;  // status word and counters
+  p.off_counters = 256;  // inside the zeroed header, after the status word
+  size_t off = kWorkspaceHeader;
   const size_t shn = (size_t)sh.S * sh.Hkv;
-  // finalize: two resident CTAs per SM and a single wave; the output CTAs take
-  // their share, the score CTAs the rest, each a multiple of 8 tiles (one per warp)
-  const long long all_pages = (long long)sh.S * sh.Hkv * sh.max_pages;
-  const long long o_ctas = (long long)sh.S * sh.Hkv * ((sh.BG + kRowsPerFinCta - 1) / kRowsPerFinCta);
-  const long long score_target = std::max<long long>(num_sms, 2LL * num_sms - o_ctas);
-  const long long fp = (all_pages + score_target - 1) / score_target;
-  const long long tile_pages = tc::kBN / sh.P;  // score CTAs start on tile boundaries
-  p.fin_pages = (int)std::max(tile_pages * 8, (fp + tile_pages * 8 - 1) / (tile_pages * 8) * (tile_pages * 8));
   p.off_part_o = off;   off = align(off + shn * p.splits * sh.BG * sh.d * 4);
   p.off_part_ml = off;  off = align(off + shn * p.splits * sh.BG * 2 * 4);
   const size_t units_per_tile = (size_t)tc::kBN / std::min(sh.P, tc::kHalfBN);
-  p.off_pagepart = off; off = align(off + shn * p.max_tiles * sh.BG * units_per_tile * 4);
-  p.off_mtile = off;    off = align(off + shn * p.max_tiles * sh.BG * 4);
+  p.off_pagepart = off; off = align(off + shn * p.max_tiles * p.bgp * units_per_tile * 4);
+  p.off_mtile = off;    off = align(off + shn * p.max_tiles * p.bgp * 4);
   p.off_scores = off;   off = align(off + shn * sh.max_pages * 4);
+  p.off_cand = off;     off = align(off + shn * p.group_ctas * p.slot_len * 8);
+  p.off_ccnt = off;     off = align(off + shn * p.group_ctas * 4);
   p.total = off;
   return p;
 }

@@ -30,6 +30,20 @@ struct WaitCtx {
   uint32_t *status;     // global status word
 };
 
+// Records a wait that gave up: the timeout bit of the status word and, for the
+// first such wait since the word was cleared, where it happened (bits 16..23 =
+// `where`, a barrier id; bits 24..31 = the waiting warp).
+__device__ __forceinline__ void note_timeout(uint32_t *status, uint32_t where) {
+  const uint32_t site = ((where & 0xffu) << 16) | ((threadIdx.x >> 5) << 24);
+  uint32_t old = *reinterpret_cast<volatile uint32_t *>(status);
+  while ((old >> 16) == 0u) {
+    const uint32_t seen = atomicCAS(status, old, old | site);
+    if (seen == old) break;
+    old = seen;
+  }
+  raise_status(status, kStatusTimeout);
+}
+
 // ------------------------------------------------------------- mbarriers ----
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -67,16 +81,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
       if (*ctx.abort) return false;
       if (global_ns() - t0 > kWaitLimitNs) {
         *ctx.abort = 1;
-        // the first wait that gave up, for diagnosis: bits 16..23 = the barrier's
-        // shared-memory address / 8 (mod 256), bits 24..31 = the waiting warp
-        const uint32_t site = (((bar >> 3) & 0xffu) << 16) | ((threadIdx.x >> 5) << 24);
-        uint32_t old = *reinterpret_cast<volatile uint32_t *>(ctx.status);
-        while ((old >> 16) == 0u) {
-          const uint32_t seen = atomicCAS(ctx.status, old, old | site);
-          if (seen == old) break;
-          old = seen;
-        }
-        raise_status(ctx.status, kStatusTimeout);
+        // bits 16..23 = the barrier's shared-memory address / 8 (mod 256)
+        note_timeout(ctx.status, (bar >> 3) & 0xffu);
         return false;
       }
     }
@@ -118,6 +124,50 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+// The same loads with an L2 cache-policy hint (a createpolicy value).
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                                 int x, int y, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(x), "r"(y), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                                 int x, int y, int z, int w, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w), "l"(pol)
+      : "memory");
+}
+// L2 policy: lines of the accesses that carry it are evicted first.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// L2 policy: lines of the accesses that carry it are evicted last.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// Global stores with an L2 cache-policy hint.
+__device__ __forceinline__ void st_hint(float *p, float a, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(a), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void st_hint(float2 *p, float2 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(v.x), "f"(v.y), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void st_hint(float4 *p, float4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w), "l"(pol)
+               : "memory");
+}
+
 // ------------------------------------------------- clusters / DSMEM ----
 // Full cluster barrier: every thread of every CTA of the cluster; release /
 // acquire order shared- and global-memory accesses across the cluster.
@@ -149,6 +199,31 @@ __device__ __forceinline__ void grid_dep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ------------------------------------------- grid-scope group barrier ----
+// The CTAs of one group (all CTAs of one launch are co-resident: cooperative
+// launch) meet on a counter in global memory.  Each CTA's thread 0 publishes the
+// CTA's writes (they precede it through a __syncthreads) and adds 1; a waiter
+// reads the counter with acquire semantics.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t arrive_gpu(uint32_t *ctr) {
+  __threadfence();
+  return atomicAdd(ctr, 1u);
+}
+// Spins until *ctr >= target; false once kWaitLimitNs has passed.
+__device__ __forceinline__ bool wait_count_geq(const uint32_t *ctr, uint32_t target) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = global_ns();
+  while (ld_acquire_gpu(ctr) < target) {
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(64);
+  }
+  return true;
+}
+
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
@@ -164,6 +239,15 @@ __device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint3
       "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           dst_cluster),
       "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+// Bulk copy (TMA engine) of `bytes` from global memory into this CTA's shared
+// memory; completes `bytes` on mbarrier `bar`.  Both addresses 16-byte aligned,
+// size a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -202,6 +286,11 @@ __device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
 }
 
 // Generic-proxy shared-memory writes made visible to the async proxy (TMA/UMMA).
+// Orders this thread's generic-proxy global accesses before later async-proxy
+// (bulk copy / TMA) accesses, and the reverse.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

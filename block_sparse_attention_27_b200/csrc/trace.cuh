@@ -29,6 +29,13 @@ static __device__ unsigned long long g_dsa_trace[dsa::kTraceCtas * dsa::kTraceEv
     asm volatile("" ::"r"((unsigned)(val)) : "memory");  \
     DSA_TRACE_EVENT(ev);                                 \
   } while (0)
+// store a raw value (a duration, a count) in the event slot instead of a timestamp
+#define DSA_TRACE_VALUE(ev, v)                                                              \
+  do {                                                                                     \
+    const unsigned cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+    if (cta_ < (unsigned)::dsa::kTraceCtas)                                                \
+      g_dsa_trace[cta_ * ::dsa::kTraceEvents + (ev)] = (unsigned long long)(v);            \
+  } while (0)
 #define DSA_TRACE_EXPORT(fn)                                                         \
   extern "C" int fn(void *host, size_t bytes) {                                     \
     if (bytes > sizeof(g_dsa_trace)) bytes = sizeof(g_dsa_trace);                   \
@@ -45,6 +52,9 @@ static __device__ unsigned long long g_dsa_trace[dsa::kTraceCtas * dsa::kTraceEv
   } while (0)
 #define DSA_TRACE_AFTER(ev, val) \
   do {                           \
+  } while (0)
+#define DSA_TRACE_VALUE(ev, v) \
+  do {                         \
   } while (0)
 #define DSA_TRACE_EXPORT(fn)
 #endif

@@ -31,7 +31,8 @@ DSA_SELECT_STATIC_SCRATCH_BYTES = 16 << 20
 # every symbol include/dsa.h declares
 EXPORTED = ("dsa_select", "dsa_sparse_attn", "dsa_select_workspace_size",
             "dsa_sparse_workspace_size", "dsa_workspace_init", "dsa_get_status",
-            "dsa_strerror", "dsa_kernels_per_call", "dsa_version", "dsa_select_static_scratch",
+            "dsa_strerror", "dsa_kernels_per_call", "dsa_select_launches", "dsa_version",
+            "dsa_select_static_scratch",
             "dsa_merge_attn")
 
 
@@ -86,13 +87,24 @@ def load(path: str = LIB_PATH):
     lib.dsa_version.argtypes = []
     lib.dsa_kernels_per_call.restype = ci
     lib.dsa_kernels_per_call.argtypes = [ci]
+    lib.dsa_select_launches.restype = ci
+    lib.dsa_select_launches.argtypes = [dims_p]
     _lib = lib
     return lib
 
 
 def kernels_per_call(pass_: int) -> int:
-    """Kernel launches per call: 0 = dsa_select, 1 = dsa_sparse_attn."""
+    """Kernel launches per call: 0 = dsa_select (groups in one launch), 1 = dsa_sparse_attn,
+    2 = dsa_merge_attn."""
     return int(load().dsa_kernels_per_call(int(pass_)))
+
+
+def select_launches(dims: dsa_dims) -> int:
+    """Kernel launches of one dsa_select call with these dims on the current device."""
+    rc = int(load().dsa_select_launches(ctypes.byref(dims)))
+    if rc < 0:
+        raise DsaError(rc, "dsa_select_launches")
+    return rc
 
 
 def strerror(code: int) -> str:

@@ -117,6 +117,11 @@ typedef struct CUstream_st *dsa_stream_t;
  * [S]); page (must equal dims->page); topk (DEVICE int32 [S], tokens); idx_out
  * (device int32 [S,Hkv,kmax]); o_out (device bf16 [S,B,Hq,d]); stream; dims;
  * cnt_out (device int32 [S,Hkv]); workspace/ws_bytes (device, see above).
+ * Launches: one cooperative kernel per dsa_select_launches(dims) groups of
+ * (sequence, KV head) whose CTAs are all resident at once (one launch when
+ * S * Hkv * ceil(B * Hq/Hkv / 128) does not exceed the SMs it may use).  The
+ * CTAs of a (sequence, KV head) wait for one another at one point, with a
+ * bounded wait (DSA_ERR_DEVICE_TIMEOUT if it gives up).
  */
 int dsa_select(const void *q_blk, const void *k_cache, const void *v_cache,
                const int32_t *n_ctx, int32_t page, const int32_t *topk,
@@ -154,7 +159,9 @@ int dsa_workspace_init(void *workspace, size_t ws_bytes, dsa_stream_t stream);
  * is left as it is (sticky).  Returns DSA_ERR_CUDA if the read fails.  After a
  * DSA_ERR_DEVICE_TIMEOUT, bits 16..31 of the word (read it directly) identify the
  * first wait that gave up: bits 16..23 its barrier's shared-memory address / 8
- * (mod 256), bits 24..31 the waiting warp. */
+ * (mod 256), or 255 for the selection pass's wait on the other CTAs of its
+ * (sequence, KV head); bits 24..31 the waiting warp.  A workspace whose call
+ * timed out must be zeroed again with dsa_workspace_init() before its next use. */
 int dsa_get_status(const void *workspace, dsa_stream_t stream);
 
 /*
@@ -165,8 +172,8 @@ int dsa_get_status(const void *workspace, dsa_stream_t stream);
  * allocate device memory at this point (for instance a plugin of an inference
  * runtime whose host hands it no workspace, or a path that runs while the
  * process's memory pool is fully reserved) cannot supply the workspace
- * dsa_select needs.  This variant launches the same three kernels as dsa_select
- * with their scratch placed in a fixed device array that the library itself
+ * dsa_select needs.  This variant launches the same kernel as dsa_select
+ * with its scratch placed in a fixed device array that the library itself
  * holds: a file-scope __device__ array of DSA_SELECT_STATIC_SCRATCH_BYTES
  * (16 MiB) per device, set aside when the CUDA module is loaded, not by an
  * allocation call.  The call allocates nothing.
@@ -185,7 +192,9 @@ int dsa_get_status(const void *workspace, dsa_stream_t stream);
  *   stream) reads it (it only reads the first word of what it is given); writing
  *   0 clears it.
  * The scratch array needs no zeroing: every word of it a call reads was written
- * earlier in the same call.
+ * earlier in the same call, except the counters of the selection pass's group
+ * wait in its first 4 KiB, which are zero when the module is loaded and which
+ * every call leaves at zero.
  *
  * Concurrency: the scratch array is one per device, shared by every call on that
  * device.  Calls on one device must not overlap in time: issue them on one
@@ -222,10 +231,16 @@ int dsa_merge_attn(const void *o_a, const float *lse_a, const void *o_b, const f
 /* Static description of a status code. */
 const char *dsa_strerror(int code);
 
-/* Number of kernel launches one call issues on its stream: pass 0 = dsa_select,
- * pass 1 = dsa_sparse_attn, pass 2 = dsa_merge_attn (DSA_ERR_INVALID_ARG otherwise).  Useful when
- * capturing calls into a CUDA graph or counting launches. */
+/* Number of kernel launches one call issues on its stream: pass 0 = dsa_select
+ * when its groups fit in one launch (dsa_select_launches() gives the count for
+ * a shape), pass 1 = dsa_sparse_attn, pass 2 = dsa_merge_attn
+ * (DSA_ERR_INVALID_ARG otherwise).  Useful when capturing calls into a CUDA
+ * graph or counting launches. */
 int dsa_kernels_per_call(int pass);
+
+/* Kernel launches of one dsa_select (or dsa_select_static_scratch) call with
+ * these dims on the current device, or a negative DSA_ERR_* code for bad dims. */
+int dsa_select_launches(const dsa_dims *dims);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int dsa_version(void);

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from block_sparse_attention_27_b200 import build as B
 from block_sparse_attention_27_b200 import dsa
@@ -130,3 +131,19 @@ def test_merge_entry_checks_on_host(lib):
     assert lib.dsa_merge_attn(ok, ok, ok, ok, ok, None, 4, 12, None) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_merge_attn(ok, ok, bad, ok, ok, None, 4, 128, None) == dsa.DSA_ERR_INVALID_ARG
     assert dsa.kernels_per_call(2) == 1
+
+
+def test_select_launches(lib):
+    """The selection pass runs its (sequence, KV head) groups in co-resident
+    launches: one for the bench shape, more when the groups outnumber the SMs
+    (148 assumed without a GPU)."""
+    if torch.cuda.is_available():
+        pytest.skip("launch counts below assume 148 SMs")
+    assert dsa.select_launches(good_dims()) == 1
+    assert dsa.select_launches(good_dims(sm_limit=37)) == 1
+    # 512 groups of one CTA: 148 per launch
+    assert dsa.select_launches(good_dims(S=64)) == 4
+    # 224 query rows per KV head: two 128-row tiles per group, 74 groups per launch
+    assert dsa.select_launches(good_dims(S=100, Hq=28, Hkv=4)) == 6
+    with pytest.raises(dsa.DsaError):
+        dsa.select_launches(good_dims(d=96))
