@@ -91,6 +91,8 @@ class Oracle:
         lib.oracle_sparse.restype = ci
         lib.oracle_sparse.argtypes = [u16p, u16p, u16p, i32p, i32p, i32p, i32p, ci, u16p, u16p,
                                       ci, ci, ci, ci, ci, ci, ci, cl, f64p, f64p]
+        lib.oracle_select_global.restype = ci
+        lib.oracle_select_global.argtypes = [f64p, i32p, i32p, ci, ci, ci, ci, ci, i32p, i32p]
         lib.oracle_num_threads.restype = ci
         lib.oracle_num_threads.argtypes = []
         self.lib = lib
@@ -132,6 +134,33 @@ class Oracle:
         if rc != ORACLE_OK:
             raise OracleError(f"oracle_select failed with status {rc}")
         return SelectResult(idx, cnt, o, lse, score, mass)
+
+    def select_global(self, q, k, v, n_ctx, topk, *, kmax, page_table=None, max_pages=None,
+                      score=None) -> SelectResult:
+        """Selection pass with the head-adaptive budget: one budget of Hkv * topk/P pages
+        per sequence shared by its KV heads (see oracle_select_global).  The page scores
+        and the prefix output are those of select(); `score` ([S, Hkv, max_pages]
+        float64) skips recomputing them."""
+        n_ctx_a = _i32(n_ctx).reshape(-1)
+        topk_a = _i32(topk).reshape(-1)
+        S = n_ctx_a.shape[0]
+        Hkv, P = _u16(k).shape[1], _u16(k).shape[2]
+        max_pages = self._max_pages(n_ctx_a, P, page_table, max_pages)
+        base = None
+        if score is None:
+            base = self.select(q, k, v, n_ctx, topk, page_table=page_table, max_pages=max_pages)
+            score = base.score
+        score = np.ascontiguousarray(score, dtype=np.float64)
+        idx = np.empty((S, Hkv, int(kmax)), np.int32)
+        cnt = np.empty((S, Hkv), np.int32)
+        I, F = ctypes.c_int32, ctypes.c_double
+        rc = self.lib.oracle_select_global(_p(score, F), _p(n_ctx_a, I), _p(topk_a, I), S, Hkv, P,
+                                           max_pages, int(kmax), _p(idx, I), _p(cnt, I))
+        if rc != ORACLE_OK:
+            raise OracleError(f"oracle_select_global failed with status {rc}")
+        if base is None:
+            return SelectResult(idx, cnt, None, None, score, None)
+        return SelectResult(idx, cnt, base.o, base.lse, score, base.mass)
 
     def sparse(self, q, k, v, n_ctx, idx, cnt, blk_k, blk_v, *, page_table=None,
                max_pages=None):
@@ -178,6 +207,10 @@ def select(*args, **kwargs) -> SelectResult:
 
 def sparse(*args, **kwargs):
     return default().sparse(*args, **kwargs)
+
+
+def select_global(*args, **kwargs) -> SelectResult:
+    return default().select_global(*args, **kwargs)
 
 
 def all_pages(n_ctx, P, Hkv, kmax=None):

@@ -216,6 +216,68 @@ int oracle_select(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 }
 
 /*
+ * Head-adaptive budget ("Step-dLLM: Adaptive Step-aware Sparse Attention for
+ * Efficient Diffusion LLM Inference", abstract: one global budget shared by the
+ * heads, so that heads whose attention is concentrated are compressed more).
+ * Reading: sequence s has one budget of Hkv * kp pages, kp = topk[s]/P being the
+ * per-head budget of the MAGE selection.  All (KV head, page) pairs of the
+ * sequence are ranked by their page score (each head's scores sum to one over its
+ * pages, so scores of different heads compare) and the best Hkv * kp pairs are
+ * kept; on equal scores the lower head wins, then the lower page.  A head may
+ * keep any number of pages, none included.
+ *   score    [S,Hkv,max_pages]   page scores (those of oracle_select)
+ *   idx_out  [S,Hkv,kmax]        each head's kept pages, ascending, -1 padded
+ *   cnt_out  [S,Hkv]             each head's count
+ * Returns ORACLE_EINVAL if a head keeps more than kmax pages.
+ */
+int oracle_select_global(const double *score, const int32_t *n_ctx, const int32_t *topk, int S,
+                         int Hkv, int P, int max_pages, int kmax, int32_t *idx_out,
+                         int32_t *cnt_out) {
+  if (S <= 0 || Hkv <= 0 || P <= 0 || max_pages <= 0 || kmax <= 0) return ORACLE_EINVAL;
+  for (int s = 0; s < S; ++s) {
+    if (n_ctx[s] <= 0 || n_ctx[s] > max_pages * P) return ORACLE_EINVAL;
+    if (topk[s] <= 0 || topk[s] % P != 0) return ORACLE_EINVAL;
+  }
+  int status = ORACLE_OK;
+  for (int s = 0; s < S; ++s) {
+    const int np = (n_ctx[s] + P - 1) / P;
+    const int total = Hkv * np;
+    const long budget = (long)Hkv * (topk[s] / P);
+    const int take = budget < total ? (int)budget : total;
+    /* a pair (h, page) is item h * np + page: the lower item wins a tie */
+    struct score_item *items = (struct score_item *)malloc(sizeof(struct score_item) * (size_t)total);
+    int *chosen = (int *)malloc(sizeof(int) * (size_t)total);
+    if (!items || !chosen) {
+      free(items); free(chosen);
+      return ORACLE_ENOMEM;
+    }
+    for (int h = 0; h < Hkv; ++h)
+      for (int lp = 0; lp < np; ++lp) {
+        items[h * np + lp].score = score[((size_t)s * Hkv + h) * max_pages + lp];
+        items[h * np + lp].page = h * np + lp;
+      }
+    qsort(items, (size_t)total, sizeof(struct score_item), by_score_then_page);
+    for (int r = 0; r < take; ++r) chosen[r] = items[r].page;
+    qsort(chosen, (size_t)take, sizeof(int), by_int); /* head-major, pages ascending */
+    int r = 0;
+    for (int h = 0; h < Hkv; ++h) {
+      int32_t *dst = idx_out + ((size_t)s * Hkv + h) * kmax;
+      int c = 0;
+      while (r < take && chosen[r] / np == h) {
+        if (c < kmax) dst[c] = chosen[r] % np;
+        ++c;
+        ++r;
+      }
+      if (c > kmax) status = ORACLE_EINVAL;
+      for (int j = c; j < kmax; ++j) dst[j] = -1;
+      cnt_out[(size_t)s * Hkv + h] = c < kmax ? c : kmax;
+    }
+    free(items); free(chosen);
+  }
+  return status;
+}
+
+/*
  * Sparse pass.  For each query row (b, j) of the block: softmax attention over
  * the valid tokens of the selected pages of KV head j/G plus the block's own B
  * tokens (keys blk_k[s,u,h], values blk_v[s,u,h], u = 0..B-1, no mask).

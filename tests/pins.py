@@ -345,8 +345,82 @@ def pin_rejects_bad_indices(orc):
         raise AssertionError(f"index list {bad} was accepted")
 
 
+# ------------------------------------------------- head-adaptive budget (Step-dLLM)
+def run_global(orc, w: W.Workload, kmax=None):
+    kmax = w.max_pages if kmax is None else kmax
+    return orc.select_global(W.bits(w.q1), W.bits(w.k_cache), W.bits(w.v_cache), w.n_ctx.numpy(),
+                             w.topk.numpy(), kmax=kmax,
+                             page_table=None if w.page_table is None else w.page_table.numpy(),
+                             max_pages=w.max_pages)
+
+
+def brute_force_global(mass: dict, s: int, Hkv: int, n: int, P: int, budget: int):
+    """Best `budget` (head, page) pairs of sequence s by page mass, by enumerating every
+    subset in lexicographic (head, page) order; ties -> the first such subset."""
+    np_ = (n + P - 1) // P
+    items = [(h, lp) for h in range(Hkv) for lp in range(np_)]
+    page_mass = {(h, lp): mass[(s, h)][lp * P:min((lp + 1) * P, n)].sum() for h, lp in items}
+    if budget >= len(items):
+        return items
+    best, best_m = None, -1.0
+    for U in itertools.combinations(items, budget):
+        m = sum(page_mass[x] for x in U)
+        if m > best_m + 1e-12:
+            best, best_m = list(U), m
+    return best
+
+
+def pin_global_brute_force(orc, seeds=(2, 3)):
+    """Head-adaptive selection equals the best (head, page) subset of the shared budget
+    found by enumerating all of them."""
+    for seed in seeds:
+        for kw in (dict(n=120, topk=32, needle_count=1), dict(n=100, topk=16, Hkv=3, Hq=6, needle_count=1)):
+            w = brute_sized(seed, **kw)
+            r = run_global(orc, w)
+            mass = token_mass_np(w)
+            best = brute_force_global(mass, 0, w.Hkv, int(w.n_ctx[0]), w.P, w.Hkv * w.kmax)
+            got = [(h, int(lp)) for h in range(w.Hkv) for lp in r.idx[0, h, :r.cnt[0, h]]]
+            assert sorted(got) == sorted(best), (seed, kw, got, best)
+            assert sum(r.cnt[0]) == w.Hkv * w.kmax
+
+
+def pin_global_one_head_is_per_head(orc):
+    """With one KV head the shared budget is that head's budget: the per-head selection."""
+    for seed in (1, 2):
+        w = brute_sized(seed, B=2, Hq=2, Hkv=1, topk=48)
+        r1, r2 = run(orc, w, kmax=w.max_pages), run_global(orc, w)
+        assert np.array_equal(r1.idx, r2.idx) and np.array_equal(r1.cnt, r2.cnt)
+
+
+def pin_global_covers_prefix(orc):
+    """A budget of at least every page of every head keeps all of them."""
+    w = small_paged(3)
+    w = W.Workload(**{**w.__dict__, "topk": torch.full((w.S,), w.max_pages * w.P, dtype=torch.int32)})
+    r = run_global(orc, w)
+    for s in range(w.S):
+        for h in range(w.Hkv):
+            assert r.idx[s, h, :r.cnt[s, h]].tolist() == list(range(w.n_pages(s)))
+
+
+def pin_global_concentrated_head(orc):
+    """A head whose attention sits on two planted pages keeps just those two; the
+    diffuse head takes the rest of the shared budget (the Step-dLLM intent)."""
+    w = brute_sized(7, n=208, topk=64, B=2, Hq=4, Hkv=2, needle_count=0)
+    qmean = f64(w.q1)[0].reshape(w.B, w.Hkv, w.G, w.d).mean(axis=(0, 2))  # [Hkv, d]
+    pages = (3, 8)
+    k = w.k_cache.float()
+    for lp in pages:
+        k[lp, 0] += 8.0 * torch.from_numpy(qmean[0]).float()
+    w.k_cache = k.to(torch.bfloat16)
+    r = run_global(orc, w)
+    assert r.idx[0, 0, :r.cnt[0, 0]].tolist() == list(pages), r.idx[0, 0, :r.cnt[0, 0]]
+    assert r.cnt[0, 1] == w.Hkv * w.kmax - len(pages)
+
+
 FAST_PINS = [pin_score_sums, pin_dense_equivalence, pin_topk_brute_force,
              pin_exact_tie_lower_index, pin_planted_needles, pin_merge_identity,
              pin_selection_output_is_prefix_attention, pin_page_table_invariance,
              pin_query_order_invariance, pin_single_row, pin_budget_covers_prefix,
-             pin_ascending_and_padding, pin_worked_example, pin_rejects_bad_indices]
+             pin_ascending_and_padding, pin_worked_example, pin_rejects_bad_indices,
+             pin_global_brute_force, pin_global_one_head_is_per_head, pin_global_covers_prefix,
+             pin_global_concentrated_head]

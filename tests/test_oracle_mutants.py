@@ -48,6 +48,12 @@ MUTANTS = [
     ("query_row_ignored", "const size_t qoff = (((size_t)s * B + b) * Hq + j) * (size_t)d;",
      "const size_t qoff = (((size_t)s * B + 0) * Hq + j) * (size_t)d;", 0),
     ("max_not_subtracted_sparse", "sum += exp(logit[t] - mx);", "sum += exp(logit[t]);", 1),
+    ("global_budget_per_head", "const long budget = (long)Hkv * (topk[s] / P);",
+     "const long budget = (long)(topk[s] / P);", 0),
+    ("global_items_head_ignored", "items[h * np + lp].score = score[((size_t)s * Hkv + h) * max_pages + lp];",
+     "items[h * np + lp].score = score[((size_t)s * Hkv + 0) * max_pages + lp];", 0),
+    ("global_pages_unsorted", "qsort(chosen, (size_t)take, sizeof(int), by_int); /* head-major",
+     "(void)by_int; /* head-major", 0),
 ]
 
 
