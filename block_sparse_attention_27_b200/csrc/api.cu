@@ -49,6 +49,8 @@ int make_shape(const dsa_dims *dims, Shape *out) {
   if ((long long)d.B * G > 256) return DSA_ERR_UNSUPPORTED;
   if ((long long)d.max_pages * d.page > (1LL << 30)) return DSA_ERR_UNSUPPORTED;
   if (d.sm_limit < 0) return DSA_ERR_INVALID_ARG;
+  if (d.head_budget != 0 && d.head_budget != 1) return DSA_ERR_INVALID_ARG;
+  if (d.head_budget && d.Hkv > dsa::kMaxHeadsAdaptive) return DSA_ERR_UNSUPPORTED;
   Shape s{};
   s.S = d.S; s.B = d.B; s.Hq = d.Hq; s.Hkv = d.Hkv; s.G = G; s.BG = d.B * G;
   s.d = d.d; s.P = d.page; s.max_pages = d.max_pages; s.kmax = d.kmax;
@@ -57,6 +59,7 @@ int make_shape(const dsa_dims *dims, Shape *out) {
   s.sl2 = (float)(1.4426950408889634 / std::sqrt((double)d.d));
   s.sm_limit = d.sm_limit;
   s.lse_out = d.lse_out;
+  s.head_budget = d.head_budget;
   *out = s;
   return DSA_OK;
 }
@@ -134,7 +137,7 @@ int dsa_select_launches(const dsa_dims *dims) {
   Shape sh;
   const int rc = make_shape(dims, &sh);
   if (rc != DSA_OK) return rc;
-  return dsa::plan_select(sh, select_sms(sh)).launches;
+  return dsa::plan_select(sh, select_sms(sh)).launches + (sh.head_budget ? dsa::kGlobalLaunches : 0);
 }
 
 size_t dsa_select_workspace_size(const dsa_dims *dims) {

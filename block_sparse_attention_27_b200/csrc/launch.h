@@ -17,6 +17,7 @@ struct Shape {
   float sl2;                  // log2(e) / sqrt(d)
   int sm_limit;               // selection pass: SMs it may hold (0 = all)
   float *lse_out;             // optional [S, B, Hq]: each row's log-sum-exp (natural log)
+  int head_budget;            // selection pass: 1 = one budget of Hkv*kp pages per sequence
 };
 
 // TMA map of a paged cache [n_phys, Hkv, P, D] viewed as rows of D bf16; boxes of
@@ -38,6 +39,10 @@ cudaError_t make_blk_tensor_map(CUtensorMap *out, const void *base, long long to
 // groups fit in one co-resident launch; see SelectPlan::launches) and by one
 // dsa_sparse_attn call.
 constexpr int kSelectLaunches = 1;
+// extra launch of the selection pass under the head-adaptive budget, and the
+// most KV heads it supports
+constexpr int kGlobalLaunches = 1;
+constexpr int kMaxHeadsAdaptive = 64;
 constexpr int kSparseLaunches = 1;
 constexpr int kMergeLaunches = 1;
 

@@ -410,13 +410,14 @@ __device__ __forceinline__ void radix_threshold(int n, int take, KeyAt key_at, T
   __syncthreads();  // sc is reused by the caller
 }
 
-// Emits (position, output slot) of the kept keys in ascending position: a
-// contiguous chunk of positions per thread, block-wide exclusive scans of the
-// counts of keys > T and == T; the slot of a kept key is
-// (greater before) + min(equal before, need_eq).
-template <class KeyAt, class Emit>
-__device__ __forceinline__ void ordered_emit(int n, uint32_t thr, uint32_t need_eq, KeyAt key_at,
-                                             Emit emit, TopkScratch &sc) {
+// Visits the positions 0..n-1 in ascending order, each thread a contiguous
+// chunk, as visit(i, before, kept): kept tells whether key i is kept (key > T, or
+// key == T among the first need_eq such positions) and before counts the kept
+// positions below i.  The counts come from block-wide exclusive scans of each
+// chunk's numbers of keys > T and == T.
+template <class KeyAt, class Visit>
+__device__ __forceinline__ void ordered_visit(int n, uint32_t thr, uint32_t need_eq, KeyAt key_at,
+                                              Visit visit, TopkScratch &sc) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = (int)blockDim.x;
   const int warps = nt >> 5;
   const int chunk = (n + nt - 1) / nt;
@@ -459,15 +460,22 @@ __device__ __forceinline__ void ordered_emit(int n, uint32_t thr, uint32_t need_
   uint32_t gt_before = g - n_gt + (warp > 0 ? sc.scan_gt[warp - 1] : 0u);
   for (int i = i0; i < i1; ++i) {
     const uint32_t key = key_at(i);
-    if (key > thr) {
-      emit(i, (int)(gt_before + min(eq_before, need_eq)));
-      ++gt_before;
-    } else if (key == thr) {
-      if (eq_before < need_eq) emit(i, (int)(gt_before + eq_before));
-      ++eq_before;
-    }
+    const bool gt = key > thr, eq = key == thr;
+    visit(i, (int)(gt_before + min(eq_before, need_eq)), gt || (eq && eq_before < need_eq));
+    gt_before += gt;
+    eq_before += eq;
   }
   __syncthreads();  // sc is reused by the caller
+}
+
+// Emits (position, output slot) of the kept keys in ascending position; the slot
+// of a kept key is the number of kept keys before it.
+template <class KeyAt, class Emit>
+__device__ __forceinline__ void ordered_emit(int n, uint32_t thr, uint32_t need_eq, KeyAt key_at,
+                                             Emit emit, TopkScratch &sc) {
+  ordered_visit(n, thr, need_eq, key_at, [&](int i, int before, bool kept) {
+    if (kept) emit(i, before);
+  }, sc);
 }
 
 // The take largest of n keys (ties to the lower position), emitted in ascending
@@ -981,13 +989,16 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   __syncthreads();
 
   // ---- 3. row statistics, page scores, local candidates ----
+  // (under the head-adaptive budget the selection is select_global_topk's: this
+  // kernel only writes the page scores)
+  const bool per_head = sh.head_budget == 0;
   int kp = topk_tokens / PAGE;
-  if (kp > sh.kmax || kp < 0 || topk_tokens % PAGE != 0) {
+  if ((per_head && kp > sh.kmax) || kp < 0 || topk_tokens % PAGE != 0) {
     if (threadIdx.x == 0 && c == 0) raise_status(a.status, kStatusBadIndex);
     kp = max(0, min(kp, sh.kmax));
   }
   const int take = min(kp, np);
-  const bool every_page = take >= np;
+  const bool every_page = take >= np || !per_head;
   const bool fast = kp <= kFastTopk;
   const int E = every_page ? 0 : (!fast ? 0 : (kp <= 32 ? 1 : (kp <= 64 ? 2 : 4)));
   merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv, [&]() {
@@ -1033,7 +1044,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     if (sc.flag) __threadfence();  // the other CTAs' candidates are visible from here on
   }
   __syncthreads();
-  if (sc.flag) {
+  if (sc.flag && per_head) {
     int32_t *out = a.idx_out + sh_idx * sh.kmax;
     const uint64_t *lists = a.cand + sh_idx * G * plan.slot_len;
     if (every_page) {
@@ -1111,6 +1122,74 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Head-adaptive budget ("Step-dLLM: Adaptive Step-aware Sparse Attention for
+// Efficient Diffusion LLM Inference", abstract): one CTA per sequence ranks the
+// (KV head, page) pairs of the sequence by the page scores select_fused wrote
+// and keeps the best Hkv * kp; pair (h, q) is position h * np + q, so ties go to
+// the lower head, then the lower page.  Each head's kept pages are written in
+// ascending order, a head keeping any number of them (none included).
+// ---------------------------------------------------------------------------
+constexpr int kGlobalThreads = 1024;
+
+__global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __grid_constant__ PartialParams pp) {
+  __shared__ TopkScratch sc;
+  __shared__ int s_base[kMaxHeadsAdaptive + 1];  // kept pairs before head h
+  const Shape &sh = pp.sh;
+  const SelectArgs &a = pp.a;
+  sm100::grid_dep_wait();  // the page scores of select_fused
+  sm100::grid_dep_launch_dependents();
+  const int s = blockIdx.x, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5, warps = (int)blockDim.x >> 5;
+  const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, sh.P, a.status, false);
+  const int np = (n + sh.P - 1) / sh.P;
+  const int topk_tokens = a.topk[s];
+  int kp = topk_tokens / sh.P;
+  if (kp < 0 || topk_tokens % sh.P != 0) {
+    if (tid == 0) raise_status(a.status, kStatusBadIndex);
+    kp = max(0, kp);
+  }
+  const int total = sh.Hkv * np;
+  const int take = (int)min((long long)sh.Hkv * kp, (long long)total);
+  const float *scores = a.scores + (size_t)s * sh.Hkv * sh.max_pages;
+  auto key_at = [&](int i) -> uint32_t {
+    const int h = i / np;
+    return score_key(__ldcg(scores + (size_t)h * sh.max_pages + (i - h * np)));
+  };
+  uint32_t thr = 0u, need_eq = (uint32_t)total;  // take == total: every pair (keys >= 0)
+  if (take == 0) {
+    thr = 0xffffffffu;  // above every key: none kept
+    need_eq = 0u;
+  } else if (take < total) {
+    radix_threshold(total, take, key_at, sc, thr, need_eq);
+  }
+  // where each head's pairs start among the kept ones
+  if (tid == 0) s_base[sh.Hkv] = take;
+  if (np == 0) {
+    for (int h = tid; h < sh.Hkv; h += blockDim.x) s_base[h] = 0;
+  } else {
+    ordered_visit(total, thr, need_eq, key_at, [&](int i, int before, bool) {
+      if (i % np == 0) s_base[i / np] = before;
+    }, sc);
+  }
+  __syncthreads();
+  int32_t *out = a.idx_out + (size_t)s * sh.Hkv * sh.kmax;
+  if (take > 0) {
+    ordered_visit(total, thr, need_eq, key_at, [&](int i, int before, bool kept) {
+      if (!kept) return;
+      const int h = i / np, pos = before - s_base[h];
+      if (pos < sh.kmax) out[(size_t)h * sh.kmax + pos] = i - h * np;
+    }, sc);
+  }
+  for (int h = warp; h < sh.Hkv; h += warps) {
+    const int cnt = s_base[h + 1] - s_base[h];
+    if (cnt > sh.kmax && lane == 0) raise_status(a.status, kStatusBadIndex);
+    const int kept = min(cnt, sh.kmax);
+    for (int j = kept + lane; j < sh.kmax; j += 32) out[(size_t)h * sh.kmax + j] = -1;
+    if (lane == 0) a.cnt_out[(size_t)s * sh.Hkv + h] = kept;
+  }
+}
+
 template <int D, int PAGE>
 cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectArgs &a,
                          cudaStream_t stream) {
@@ -1149,6 +1228,15 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
     pp.group0 = g0;
     cfg.gridDim = dim3(std::min(plan.groups_per_launch, groups - g0) * plan.group_ctas, 1, 1);
     err = cudaLaunchKernelEx(&cfg, kern, pp, kmap, vmap, kmap4, vmap4);
+    if (err != cudaSuccess) return err;
+  }
+  if (sh.head_budget) {  // the selection over all KV heads of each sequence
+    cfg.attrs = attrs + 1;  // programmatic dependent only
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(sh.S, 1, 1);
+    cfg.blockDim = dim3(kGlobalThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    err = cudaLaunchKernelEx(&cfg, select_global_topk, pp);
     if (err != cudaSuccess) return err;
   }
   return cudaGetLastError();

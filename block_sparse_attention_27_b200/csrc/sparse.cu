@@ -73,7 +73,7 @@ struct SparsePolicy {
   const int2 *tab;              // shared: (lp, phys) per entry of this CTA, phys < 0 = unusable
   const uint64_t *masks;        // shared: key mask of each page tile
   uint32_t tab_off, mask_off;   // byte offsets in the aligned shared memory
-  int lp_spec;                  // warp 0: idx[s, h, c*ppc + lane], loaded with idx_cnt
+  int lp_spec;                  // warp 0: idx[s, h, c*ppc + lane], loaded with idx_cnt (-2: not this slice)
   long long n_phys, phys0;
   int Hkv, h, G, Hq, B, BG, s, n, np, e_begin, e_end, sel_tiles, row_base;
   float sl2;
@@ -93,10 +93,10 @@ struct SparsePolicy {
     masks = mk;
     if (threadIdx.x >= 32) return;
     const int lane = threadIdx.x;
-    // e_begin == c * ppc whenever the slice is not empty, so entry i = lane of the
-    // first pass is the one loaded speculatively
+    // e_begin == c * ppc whenever the slice is not empty and lp_spec != -2, so
+    // entry i = lane of the first pass is then the one loaded speculatively
     for (int i = lane; i < e_end - e_begin; i += 32) {
-      const int lp = i == lane ? lp_spec : idx_row[e_begin + i];
+      const int lp = (i == lane && lp_spec != -2) ? lp_spec : idx_row[e_begin + i];
       const int2 v = resolve_lp(lp);
       if (v.y < 0) raise_status(status, kStatusBadIndex);
       t[i] = v;
@@ -279,8 +279,13 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     cnt = max(0, min(cnt, sh.kmax));
   }
   if (threadIdx.x == 0) DSA_TRACE_AFTER(34, cnt + n);
-  const int e_begin = blk_cta ? cnt : min(cnt, c * plan.ppc);
-  const int e_end = blk_cta ? cnt : min(cnt, (c + 1) * plan.ppc);
+  // the page CTAs split this head's cnt pages evenly, in whole tiles (counts
+  // differ per head under the head-adaptive budget); ppc_eff = plan.ppc when
+  // cnt = kmax, and then the speculative idx load above is this CTA's slice
+  const int ppc_eff = min(plan.ppc, ((cnt + C - 2) / (C - 1) + kPagesPerTile - 1) / kPagesPerTile * kPagesPerTile);
+  const int e_begin = blk_cta ? cnt : min(cnt, c * ppc_eff);
+  const int e_end = blk_cta ? cnt : min(cnt, (c + 1) * ppc_eff);
+  if (ppc_eff != plan.ppc) lp_spec = -2;  // not this slice's: prepare() loads it again
   const int sel_tiles = (e_end - e_begin + kPagesPerTile - 1) / kPagesPerTile;
   const int num_tiles = sel_tiles + (blk_cta ? plan.blk_tiles : 0);
 

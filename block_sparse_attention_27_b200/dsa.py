@@ -47,7 +47,8 @@ class dsa_dims(ctypes.Structure):
                 ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32), ("page", ctypes.c_int32),
                 ("max_pages", ctypes.c_int32), ("kmax", ctypes.c_int32),
                 ("n_phys", ctypes.c_int64), ("page_table", ctypes.c_void_p),
-                ("sm_limit", ctypes.c_int32), ("lse_out", ctypes.c_void_p)]
+                ("sm_limit", ctypes.c_int32), ("lse_out", ctypes.c_void_p),
+                ("head_budget", ctypes.c_int32)]
 
 
 _lib = None
@@ -121,9 +122,10 @@ def _stream(stream):
 
 
 def make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table=None,
-              sm_limit=0) -> dsa_dims:
+              sm_limit=0, head_budget=0) -> dsa_dims:
     return dsa_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys,
-                    None if page_table is None else page_table.data_ptr(), int(sm_limit), None)
+                    None if page_table is None else page_table.data_ptr(), int(sm_limit), None,
+                    int(head_budget))
 
 
 def _with_lse(dims: dsa_dims, lse_out) -> dsa_dims:
@@ -136,12 +138,14 @@ def _with_lse(dims: dsa_dims, lse_out) -> dsa_dims:
     return d
 
 
-def dims_for(q_blk, k_cache, max_pages, kmax, page_table=None, sm_limit=0) -> dsa_dims:
+def dims_for(q_blk, k_cache, max_pages, kmax, page_table=None, sm_limit=0,
+             head_budget=0) -> dsa_dims:
     S, B, Hq, d = q_blk.shape
     n_phys, Hkv, page, d2 = k_cache.shape
     if d2 != d:
         raise ValueError("q_blk and k_cache disagree on the head dimension")
-    return make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table, sm_limit)
+    return make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table, sm_limit,
+                     head_budget)
 
 
 def _check(t, name, dtype, ndim=None):
@@ -265,7 +269,9 @@ def dsa_merge_attn(o_a, lse_a, o_b, lse_b, o_out, lse_out=None, stream=None):
 class DeviceWorkload:
     """A workload's tensors on the GPU plus the dims, outputs and workspaces of both passes."""
 
-    def __init__(self, w, device="cuda", sm_limit=0):
+    def __init__(self, w, device="cuda", sm_limit=0, head_budget=0):
+        """head_budget=1: one budget of Hkv*kp pages per sequence shared by its KV heads;
+        idx rows then hold up to min(max_pages, Hkv*kp) pages."""
         self.w = w
         dev = torch.device(device)
         self.q1 = w.q1.to(dev)
@@ -276,9 +282,12 @@ class DeviceWorkload:
         self.n_ctx = w.n_ctx.to(dev)
         self.topk = w.topk.to(dev)
         self.page_table = None if w.page_table is None else w.page_table.to(dev)
-        self.dims = dims_for(self.q1, self.k_cache, w.max_pages, w.kmax, self.page_table, sm_limit)
+        kmax = min(w.max_pages, w.Hkv * w.kmax) if head_budget else w.kmax
+        self.kmax = kmax
+        self.dims = dims_for(self.q1, self.k_cache, w.max_pages, kmax, self.page_table, sm_limit,
+                             head_budget)
         S, Hkv = w.S, w.Hkv
-        self.idx = torch.full((S, Hkv, w.kmax), -1, dtype=torch.int32, device=dev)
+        self.idx = torch.full((S, Hkv, kmax), -1, dtype=torch.int32, device=dev)
         self.cnt = torch.zeros((S, Hkv), dtype=torch.int32, device=dev)
         self.o_sel = torch.zeros_like(self.q1)
         self.o_sp = torch.zeros_like(self.q1)

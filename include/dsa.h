@@ -97,6 +97,15 @@ typedef struct dsa_dims {
                          receives these dims stores, per query row, the natural log of the sum
                          of exp(q.k / sqrt(d)) over the keys it attends to (-inf for none),
                          so that two attention results can be merged (dsa_merge_attn). */
+  int32_t head_budget; /* selection pass: 0 = kp = topk[s]/page pages per KV head (MAGE);
+                         1 = one budget of Hkv*kp pages per sequence shared by its KV heads
+                         (head-adaptive budget, Step-dLLM page, abstract): all (KV head, page)
+                         pairs of the sequence are ranked by page score, ties going to the
+                         lower head, then the lower page, so a head whose attention is
+                         concentrated keeps fewer pages; a head may keep none.  idx_out then
+                         holds a different count per head (cnt_out); kmax must hold every
+                         head's count (min(max_pages, Hkv*kp) always does), else the call
+                         reports DSA_ERR_BAD_INDEX and keeps that head's first kmax pages. */
 } dsa_dims;
 
 /* cudaStream_t without including the CUDA headers. */
@@ -112,7 +121,8 @@ typedef struct CUstream_st *dsa_stream_t;
  *     each page, and the kp = topk[s]/page pages with the largest sums are kept;
  *     on equal sums the lower page index wins.  idx_out receives them in
  *     ascending order, padded with -1; cnt_out receives min(kp, pages of the
- *     prefix).  Requires topk[s]/page <= kmax.
+ *     prefix).  Requires topk[s]/page <= kmax.  With dims->head_budget = 1 the
+ *     kp-per-head cut is replaced by the head-adaptive budget (see dsa_dims).
  * Arguments: q_blk, k_cache, v_cache (bf16, layouts above); n_ctx (device int32
  * [S]); page (must equal dims->page); topk (DEVICE int32 [S], tokens); idx_out
  * (device int32 [S,Hkv,kmax]); o_out (device bf16 [S,B,Hq,d]); stream; dims;

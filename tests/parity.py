@@ -64,3 +64,38 @@ def check_output(gpu_o: torch.Tensor, ref: np.ndarray, what: str,
     mx, mean = float(err.max()), float(err.mean())
     assert mx <= max_abs and mean <= mean_abs, f"{what}: max {mx:.3e} mean {mean:.3e}"
     return mx, mean
+
+
+def check_global_selection(gpu_idx, gpu_cnt, orc, n_pages, kp_of, rel=TIE_REL):
+    """Head-adaptive budget: per sequence, the kept (KV head, page) pairs.  Bit-exact
+    unless the oracle's K-th and (K+1)-th pair scores (K = Hkv * kp) are within `rel`;
+    then pairs in the window W = {|S - s_K| <= rel * s_K} may go either way, the number
+    kept must be K and every pair outside W must agree.  Returns the windowed count."""
+    S, Hkv, _ = gpu_idx.shape
+    windowed = 0
+    for s in range(S):
+        np_ = n_pages[s]
+        got, want = set(), set()
+        for h in range(Hkv):
+            c = int(gpu_cnt[s, h])
+            g = gpu_idx[s, h]
+            assert np.all(g[c:] == -1), (s, h, "padding")
+            assert np.all(np.diff(g[:c]) > 0), (s, h, "ascending")
+            assert np.all((g[:c] >= 0) & (g[:c] < np_)), (s, h, "range")
+            got |= {(h, int(q)) for q in g[:c]}
+            want |= {(h, int(q)) for q in orc.idx[s, h, :orc.cnt[s, h]]}
+        total = Hkv * np_
+        K = min(Hkv * kp_of[s], total)
+        assert len(got) == K, (s, len(got), K)
+        if K == total or got == want:
+            assert got == want, (s, sorted(got ^ want))
+            continue
+        sc = orc.score[s, :, :np_].reshape(-1)          # pair (h, q) at h * np + q
+        order = np.lexsort((np.arange(total), -sc))
+        s_k, s_k1 = sc[order[K - 1]], sc[order[K]]
+        assert s_k - s_k1 <= rel * s_k, (s, sorted(got ^ want))
+        windowed += 1
+        W = {(int(i) // np_, int(i) % np_) for i in np.nonzero(np.abs(sc - s_k) <= rel * s_k)[0]}
+        assert (want - W) <= got, s
+        assert not ((got - want) - W), s
+    return windowed

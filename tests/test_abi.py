@@ -56,6 +56,8 @@ def good_dims(**kw):
     (dict(B=65, Hq=32, Hkv=8), dsa.DSA_ERR_UNSUPPORTED),  # B*G = 260 > 256
     (dict(kmax=0), dsa.DSA_ERR_INVALID_ARG),
     (dict(S=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(head_budget=2), dsa.DSA_ERR_INVALID_ARG),
+    (dict(head_budget=1, Hq=128, Hkv=128, B=1), dsa.DSA_ERR_UNSUPPORTED),  # more KV heads than supported
 ])
 def test_bad_dims_rejected_on_host(lib, kw, code):
     dims = good_dims(**kw)
