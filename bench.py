@@ -438,7 +438,21 @@ def _run_ours(args, world, rank, local, dsa):
     for i in range(3):
         exact_extra(i)
     exact_us = 1e3 * timed(exact_extra, 20, torch.cuda.current_stream())
-    del dw, qs
+    # head-adaptive budget (Step-dLLM): one budget of Hkv*kp pages per sequence shared
+    # by its KV heads; its selection pass and a sparse step on the ragged per-head
+    # counts, beside a per-head sparse step timed the same way (eager launches)
+    cur = torch.cuda.current_stream()
+    dwh = dsa.DeviceWorkload(w, head_budget=1)
+    for i in range(3):
+        dwh.select()
+    hb_sel_ms = timed(lambda i: dwh.select(), 20, cur)
+    for i in range(3):
+        dwh.sparse(dwh.q1, dwh.blk_k1, dwh.blk_v1)
+        dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1)
+    hb_sp_us = 1e3 * timed(lambda i: dwh.sparse(dwh.q1, dwh.blk_k1, dwh.blk_v1), 50, cur)
+    ph_sp_us = 1e3 * timed(lambda i: dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1), 50, cur)
+    hb_cnt = dwh.cnt.cpu().numpy()
+    del dw, dwh, qs
 
     if rank != 0:
         return
@@ -486,6 +500,13 @@ def _run_ours(args, world, rank, local, dsa):
                    "reused_step1_min": round(float(np.min(rec_reused[1:])), 4),
                    "anchor_every_8_mean": round(float(np.mean(rec_anchor8[1:])), 4)},
         "exact_step1_extra_us": round(exact_us, 2),
+        "head_budget": {"what": "one budget of Hkv*kp pages per sequence shared by its KV heads "
+                                "(dsa_dims.head_budget = 1); eager launches",
+                        "select_pass_ms": round(hb_sel_ms, 4),
+                        "sparse_step_us": round(hb_sp_us, 2),
+                        "per_head_sparse_step_us": round(ph_sp_us, 2),
+                        "pages_per_head_min": int(hb_cnt.min()),
+                        "pages_per_head_max": int(hb_cnt.max())},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)

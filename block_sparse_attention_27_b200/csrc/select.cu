@@ -1129,18 +1129,87 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // and keeps the best Hkv * kp; pair (h, q) is position h * np + q, so ties go to
 // the lower head, then the lower page.  Each head's kept pages are written in
 // ascending order, a head keeping any number of them (none included).
+//
+// Fast path (positions <= kGlobalBits, candidates <= kGlobalCand):
+//   1. the range of the keys (one pass, coalesced 16-byte loads), then a
+//      histogram of 4096 equal bins over it gives the bin holding the
+//      take-th largest key; while that bin holds too many keys, a histogram
+//      over the bin narrows it; t0 = the lower edge of the bin found;
+//   2. the keys >= t0 are compacted into shared memory with their positions,
+//      and an exact radix select among them gives T and the number of keys == T
+//      to keep;
+//   3. bitmaps over the positions: keys > T kept, keys == T kept in ascending
+//      position until need_eq of them;
+//   4. warp h writes head h's kept pages (its stretch of the bitmap) in order.
+// Otherwise every pass reads the keys from L2 (radix select and two ordered
+// visits).
 // ---------------------------------------------------------------------------
+// Calls f(key, position) for every (KV head, page) pair of a sequence, position
+// h * np + q; rows of the score array are max_pages apart.  16-byte loads, eight
+// per thread in flight, when the rows are 16-byte aligned.
+template <class F>
+__device__ __forceinline__ void for_each_pair(const float *scores, int max_pages, int Hkv, int np, F f) {
+  const int nt = (int)blockDim.x;
+  if ((max_pages & 3) == 0) {
+    const int nv = (np + 3) >> 2, tot = Hkv * nv;
+    for (int v0 = threadIdx.x; v0 < tot; v0 += 8 * nt) {
+      float4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int v = v0 + u * nt;
+        if (v < tot) {
+          const int h = v / nv, j = v - h * nv;
+          x[u] = __ldcg(reinterpret_cast<const float4 *>(scores + (size_t)h * max_pages) + j);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int v = v0 + u * nt;
+        if (v < tot) {
+          const int h = v / nv, j = v - h * nv;
+          const float e[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (4 * j + c < np) f(score_key(e[c]), h * np + 4 * j + c);
+        }
+      }
+    }
+  } else {
+    const int tot = Hkv * np;
+    for (int i0 = threadIdx.x; i0 < tot; i0 += 8 * nt) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * nt;
+        if (i < tot) {
+          const int h = i / np;
+          x[u] = __ldcg(scores + (size_t)h * max_pages + (i - h * np));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (i0 + u * nt < tot) f(score_key(x[u]), i0 + u * nt);
+    }
+  }
+}
+
 constexpr int kGlobalThreads = 1024;
+constexpr int kGlobalBits = 1 << 18;       // positions the bitmaps cover (2 x 32 KB)
+constexpr int kGlobalCand = 8192;          // candidates held in shared memory (64 KB)
+constexpr int kGlobalHistBins = 4096;
+constexpr int kGlobalSmem = 2 * (kGlobalBits / 8) + kGlobalCand * 8 + kGlobalHistBins * 4;
 
 __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __grid_constant__ PartialParams pp) {
+  extern __shared__ __align__(16) unsigned char gsm[];
   __shared__ TopkScratch sc;
   __shared__ int s_base[kMaxHeadsAdaptive + 1];  // kept pairs before head h
+  __shared__ uint32_t s_ncand, s_bin, s_above;
   const Shape &sh = pp.sh;
   const SelectArgs &a = pp.a;
   sm100::grid_dep_wait();  // the page scores of select_fused
   sm100::grid_dep_launch_dependents();
-  const int s = blockIdx.x, tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5, warps = (int)blockDim.x >> 5;
+  const int s = blockIdx.x, tid = threadIdx.x, nt = (int)blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, warps = nt >> 5;
   const int n = clamp_prefix(a.n_ctx[s], sh.max_pages, sh.P, a.status, false);
   const int np = (n + sh.P - 1) / sh.P;
   const int topk_tokens = a.topk[s];
@@ -1152,10 +1221,211 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
   const int total = sh.Hkv * np;
   const int take = (int)min((long long)sh.Hkv * kp, (long long)total);
   const float *scores = a.scores + (size_t)s * sh.Hkv * sh.max_pages;
+  int32_t *out = a.idx_out + (size_t)s * sh.Hkv * sh.kmax;
   auto key_at = [&](int i) -> uint32_t {
     const int h = i / np;
     return score_key(__ldcg(scores + (size_t)h * sh.max_pages + (i - h * np)));
   };
+  // per head: count, padding, overflow report (s_base complete)
+  auto finish_counts = [&]() {
+    for (int h = warp; h < sh.Hkv; h += warps) {
+      const int cnt = s_base[h + 1] - s_base[h];
+      if (cnt > sh.kmax && lane == 0) raise_status(a.status, kStatusBadIndex);
+      const int kept = min(cnt, sh.kmax);
+      for (int j = kept + lane; j < sh.kmax; j += 32) out[(size_t)h * sh.kmax + j] = -1;
+      if (lane == 0) a.cnt_out[(size_t)s * sh.Hkv + h] = kept;
+    }
+  };
+
+  uint32_t *keep = reinterpret_cast<uint32_t *>(gsm);                   // [kGlobalBits / 32]
+  uint32_t *eqb = keep + kGlobalBits / 32;                               // [kGlobalBits / 32]
+  uint2 *cand = reinterpret_cast<uint2 *>(eqb + kGlobalBits / 32);       // [kGlobalCand] (key, position)
+  uint32_t *hist = reinterpret_cast<uint32_t *>(cand + kGlobalCand);     // [kGlobalHistBins]
+  constexpr int kHist = kGlobalHistBins;
+  bool fast = total <= kGlobalBits && take > 0 && take < total;
+  uint32_t t0 = 0u;  // candidates: every key >= t0
+  if (fast) {
+    // 1. the key range holding the take-th largest key: the range of all keys
+    //    (one pass), then histograms of 4096 equal bins over the current range,
+    //    narrowed to the bin that holds it while that bin has too many keys
+    uint32_t kmn = 0xffffffffu, kmx = 0u;
+    for_each_pair(scores, sh.max_pages, sh.Hkv, np, [&](uint32_t key, int) {
+      kmn = min(kmn, key);
+      kmx = max(kmx, key);
+    });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+      kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+    }
+    if (lane == 0) {
+      sc.scan_eq[warp] = kmn;
+      sc.scan_gt[warp] = kmx;
+    }
+    __syncthreads();
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int w = 0; w < warps; ++w) {
+      lo = min(lo, sc.scan_eq[w]);
+      hi = max(hi, sc.scan_gt[w]);
+    }
+    __syncthreads();  // (sc is reused)
+    uint32_t above = 0u;  // keys above the current range
+    for (int level = 0; level < 4; ++level) {
+      const uint32_t width = (uint32_t)(((unsigned long long)(hi - lo) + kHist) / kHist);  // >= 1
+      for (int i = tid; i < kHist; i += nt) hist[i] = 0u;
+      if (tid == 0) {
+        s_bin = 0u;
+        s_above = 0xffffffffu;  // (set below: some bin always holds the take-th key)
+      }
+      __syncthreads();
+      for_each_pair(scores, sh.max_pages, sh.Hkv, np, [&](uint32_t key, int) {
+        if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) / width], 1u);
+      });
+      __syncthreads();
+      // the bin of the take-th largest key: warp 0 scans from the top
+      if (warp == 0) {
+        constexpr int kPer = kHist / 32;
+        uint32_t local = 0;
+        for (int j = 0; j < kPer; ++j) local += hist[kHist - 1 - (lane * kPer + j)];
+        uint32_t incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const uint32_t before = above + incl - local;
+        if (before < (uint32_t)take && (uint32_t)take <= above + incl) {
+          uint32_t cum = before;
+          for (int j = 0; j < kPer; ++j) {
+            const int bin = kHist - 1 - (lane * kPer + j);
+            if (cum + hist[bin] >= (uint32_t)take) {
+              s_bin = (uint32_t)bin;
+              s_above = cum + hist[bin];  // keys >= the bin's lower edge
+              break;
+            }
+            cum += hist[bin];
+          }
+        }
+      }
+      __syncthreads();
+      const uint32_t b = s_bin;
+      t0 = lo + b * width;
+      if (s_above <= (uint32_t)kGlobalCand || width == 1u) break;
+      above = s_above - hist[b];
+      hi = (uint32_t)min((unsigned long long)hi, (unsigned long long)t0 + width - 1u);
+      lo = t0;
+      __syncthreads();  // (hist is cleared for the next level)
+    }
+    fast = s_above <= (uint32_t)kGlobalCand;
+  }
+  if (fast) {
+    // 2. candidates: every key >= t0, with its position
+    if (tid == 0) s_ncand = 0u;
+    __syncthreads();
+    for_each_pair(scores, sh.max_pages, sh.Hkv, np, [&](uint32_t key, int pos) {
+      if (key >= t0) {
+        const uint32_t slot = atomicAdd(&s_ncand, 1u);
+        if (slot < (uint32_t)kGlobalCand) cand[slot] = make_uint2(key, (uint32_t)pos);
+      }
+    });
+    for (int w = tid; w < (total + 31) / 32; w += nt) {
+      keep[w] = 0u;
+      eqb[w] = 0u;
+    }
+    __syncthreads();
+    const int nc = (int)min(s_ncand, (uint32_t)kGlobalCand);
+    uint32_t thr = 0u, need_eq = 0u;
+    if (take < nc) {
+      radix_threshold(nc, take, [&](int i) -> uint32_t { return cand[i].x; }, sc, thr, need_eq);
+    } else {  // (every candidate is kept)
+      thr = 0u;
+      need_eq = (uint32_t)nc;
+    }
+    // 3. bitmaps: keys > T kept; keys == T in ascending position until need_eq
+    for (int i = tid; i < nc; i += nt) {
+      const uint2 c = cand[i];
+      if (c.x > thr) atomicOr(&keep[c.y >> 5], 1u << (c.y & 31));
+      else if (c.x == thr) atomicOr(&eqb[c.y >> 5], 1u << (c.y & 31));
+    }
+    __syncthreads();
+    {
+      const int words = (total + 31) / 32;
+      const int chunk = (words + nt - 1) / nt;
+      const int w0 = min(words, tid * chunk), w1 = min(words, w0 + chunk);
+      uint32_t mine = 0;
+      for (int w = w0; w < w1; ++w) mine += __popc(eqb[w]);
+      uint32_t incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (lane == 31) sc.scan_eq[warp] = incl;
+      __syncthreads();
+      if (warp == 0) {
+        uint32_t we = lane < warps ? sc.scan_eq[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t v = __shfl_up_sync(0xffffffffu, we, o);
+          if (lane >= o) we += v;
+        }
+        sc.scan_eq[lane] = we;
+      }
+      __syncthreads();
+      uint32_t before = incl - mine + (warp > 0 ? sc.scan_eq[warp - 1] : 0u);
+      for (int w = w0; w < w1; ++w) {
+        uint32_t bits = eqb[w];
+        while (bits) {
+          const int b = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          if (before < need_eq) keep[w] |= 1u << b;
+          ++before;
+        }
+      }
+    }
+    __syncthreads();
+    // 4. warp h: head h's kept pages in ascending order
+    for (int h = warp; h < sh.Hkv; h += warps) {
+      const int p0 = h * np, p1 = p0 + np;
+      int cnt = 0;
+      for (int wb = p0 >> 5; wb <= (p1 - 1) >> 5; wb += 32) {
+        const int w = wb + lane;
+        uint32_t bits = 0u;
+        if (w <= (p1 - 1) >> 5) {
+          bits = keep[w];
+          const int lo = max(p0 - w * 32, 0), hi = min(p1 - w * 32, 32);  // bits [lo, hi) of this head
+          const uint32_t mhi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+          bits &= mhi & ~((1u << lo) - 1u);
+        }
+        const int c = __popc(bits);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int pos = cnt + incl - c;
+        while (bits) {
+          const int b = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          if (pos < sh.kmax) out[(size_t)h * sh.kmax + pos] = w * 32 + b - p0;
+          ++pos;
+        }
+        cnt += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) s_base[h + 1] = cnt;  // (a count here; prefix below)
+    }
+    __syncthreads();
+    if (tid == 0) {
+      s_base[0] = 0;
+      for (int h = 0; h < sh.Hkv; ++h) s_base[h + 1] += s_base[h];
+    }
+    __syncthreads();
+    finish_counts();
+    return;
+  }
+
+  // general path: every pass reads the keys from L2
   uint32_t thr = 0u, need_eq = (uint32_t)total;  // take == total: every pair (keys >= 0)
   if (take == 0) {
     thr = 0xffffffffu;  // above every key: none kept
@@ -1163,7 +1433,6 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
   } else if (take < total) {
     radix_threshold(total, take, key_at, sc, thr, need_eq);
   }
-  // where each head's pairs start among the kept ones
   if (tid == 0) s_base[sh.Hkv] = take;
   if (np == 0) {
     for (int h = tid; h < sh.Hkv; h += blockDim.x) s_base[h] = 0;
@@ -1173,7 +1442,6 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
     }, sc);
   }
   __syncthreads();
-  int32_t *out = a.idx_out + (size_t)s * sh.Hkv * sh.kmax;
   if (take > 0) {
     ordered_visit(total, thr, need_eq, key_at, [&](int i, int before, bool kept) {
       if (!kept) return;
@@ -1181,13 +1449,7 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
       if (pos < sh.kmax) out[(size_t)h * sh.kmax + pos] = i - h * np;
     }, sc);
   }
-  for (int h = warp; h < sh.Hkv; h += warps) {
-    const int cnt = s_base[h + 1] - s_base[h];
-    if (cnt > sh.kmax && lane == 0) raise_status(a.status, kStatusBadIndex);
-    const int kept = min(cnt, sh.kmax);
-    for (int j = kept + lane; j < sh.kmax; j += 32) out[(size_t)h * sh.kmax + j] = -1;
-    if (lane == 0) a.cnt_out[(size_t)s * sh.Hkv + h] = kept;
-  }
+  finish_counts();
 }
 
 template <int D, int PAGE>
@@ -1233,9 +1495,11 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
   if (sh.head_budget) {  // the selection over all KV heads of each sequence
     cfg.attrs = attrs + 1;  // programmatic dependent only
     cfg.numAttrs = 1;
+    err = set_smem_once<select_global_topk>(kGlobalSmem);
+    if (err != cudaSuccess) return err;
     cfg.gridDim = dim3(sh.S, 1, 1);
     cfg.blockDim = dim3(kGlobalThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = kGlobalSmem;
     err = cudaLaunchKernelEx(&cfg, select_global_topk, pp);
     if (err != cudaSuccess) return err;
   }

@@ -92,3 +92,19 @@ def test_head_budget_launches(dsa_mod):
     assert dsa_mod.select_launches(dw.dims) == 2
     dw1 = dsa_mod.DeviceWorkload(w)
     assert dsa_mod.select_launches(dw1.dims) == 1
+
+
+@pytest.mark.parametrize("n,Hkv,path", [(1000, 2, "staged candidates"), (20000, 8, "keys from L2")])
+def test_head_budget_all_ties(dsa_mod, n, Hkv, path):
+    """All keys zero: every full page of every head has the same score, bit for bit,
+    on both sides.  The shared budget then goes to the lowest (head, page) pairs:
+    head 0 takes it all and the other heads keep nothing (the sparse pass then
+    attends to the block alone for them).  Covers both selection paths."""
+    w = W.make("tiny", 3, n=n, topk=256, B=4, Hq=2 * Hkv, Hkv=Hkv, d=64, needle_count=0)
+    w.k_cache = torch.zeros_like(w.k_cache)
+    dw, ref = run_global_case(dsa_mod, w)
+    got = dw.idx.cpu().numpy()
+    K = Hkv * (256 // w.P)
+    assert int(dw.cnt[0, 0]) == K and got[0, 0, :K].tolist() == list(range(K))
+    assert dw.cnt[0, 1:].sum().item() == 0
+    assert np.array_equal(got, ref.idx) and np.array_equal(dw.cnt.cpu().numpy(), ref.cnt)
