@@ -93,6 +93,11 @@ class Oracle:
                                       ci, ci, ci, ci, ci, ci, ci, cl, f64p, f64p]
         lib.oracle_select_global.restype = ci
         lib.oracle_select_global.argtypes = [f64p, i32p, i32p, ci, ci, ci, ci, ci, i32p, i32p]
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        lib.oracle_sparse_losa.restype = ci
+        lib.oracle_sparse_losa.argtypes = [u16p, u16p, u16p, i32p, i32p, i32p, i32p, ci, u16p, u16p,
+                                           u8p, u16p, f64p, ci, ci, ci, ci, ci, ci, ci, cl,
+                                           f64p, f64p, f64p, f64p]
         lib.oracle_num_threads.restype = ci
         lib.oracle_num_threads.argtypes = []
         self.lib = lib
@@ -187,6 +192,38 @@ class Oracle:
         return o, lse
 
 
+    def sparse_losa(self, q, k, v, n_ctx, idx, cnt, blk_k, blk_v, active, cache_o, cache_lse, *,
+              page_table=None, max_pages=None):
+        """Sparse pass reusing the prefix part of stable tokens (see oracle_sparse_losa).
+        active [S, B] bool; cache_o [S, B, Hq, d] bf16 bits; cache_lse [S, B, Hq] (natural log).
+        Returns (o, lse, cache_o_new, cache_lse_new), all float64."""
+        q, k, v = _u16(q), _u16(k), _u16(v)
+        blk_k, blk_v = _u16(blk_k), _u16(blk_v)
+        S, B, Hq, d = q.shape
+        n_phys, Hkv, P, _ = k.shape
+        n_ctx = _i32(n_ctx).reshape(S)
+        max_pages = self._max_pages(n_ctx, P, page_table, max_pages)
+        idx = _i32(idx)
+        cnt = _i32(cnt).reshape(S, Hkv)
+        kmax = idx.shape[-1]
+        pt = _i32(page_table) if page_table is not None else None
+        act = np.ascontiguousarray(np.asarray(active).reshape(S, B).astype(np.uint8))
+        co = _u16(cache_o)
+        cl = np.ascontiguousarray(np.asarray(cache_lse, dtype=np.float64).reshape(S, B, Hq))
+        o = np.empty((S, B, Hq, d), np.float64)
+        lse = np.empty((S, B, Hq), np.float64)
+        co_new = np.empty((S, B, Hq, d), np.float64)
+        cl_new = np.empty((S, B, Hq), np.float64)
+        I, F, U, U8 = ctypes.c_int32, ctypes.c_double, ctypes.c_uint16, ctypes.c_uint8
+        rc = self.lib.oracle_sparse_losa(
+            _p(q, U), _p(k, U), _p(v, U), _p(pt, I), _p(n_ctx, I), _p(idx, I), _p(cnt, I), kmax,
+            _p(blk_k, U), _p(blk_v, U), _p(act, U8), _p(co, U), _p(cl, F), S, B, Hq, Hkv, d, P,
+            max_pages, n_phys, _p(o, F), _p(lse, F), _p(co_new, F), _p(cl_new, F))
+        if rc != ORACLE_OK:
+            raise OracleError(f"oracle_sparse_losa failed with status {rc}")
+        return o, lse, co_new, cl_new
+
+
 _default: Oracle | None = None
 
 
@@ -211,6 +248,10 @@ def sparse(*args, **kwargs):
 
 def select_global(*args, **kwargs) -> SelectResult:
     return default().select_global(*args, **kwargs)
+
+
+def sparse_losa(*args, **kwargs):
+    return default().sparse_losa(*args, **kwargs)
 
 
 def all_pages(n_ctx, P, Hkv, kmax=None):

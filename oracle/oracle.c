@@ -374,3 +374,143 @@ int oracle_sparse(const uint16_t *q, const uint16_t *k, const uint16_t *v,
   }
   return status;
 }
+
+/*
+ * Sparse pass with reuse of the prefix part for stable tokens ("LoSA: Locality
+ * Aware Sparse Attention for Block-Wise Diffusion Language Models", abstract:
+ * cached prefix-attention results are reused for stable tokens and sparse
+ * attention is run only for active tokens).  Reading: a query row (b, j) splits
+ * its attention into the prefix part (the valid tokens of the selected pages)
+ * and the block part (the block's own B tokens), each a normalised output with
+ * its log-sum-exp.  For an active token (active[s,b] != 0) the prefix part is
+ * computed and written to cache_o_out / cache_lse_out; for a stable token it is
+ * taken from cache_o_in (bf16 bits) / cache_lse_in and passed through.  The block
+ * part is always computed.  The row's output merges the two:
+ *   lse = log(exp(lse_p) + exp(lse_b)),  o = exp(lse_p - lse) o_p + exp(lse_b - lse) o_b,
+ * an empty part having lse = -inf and o = 0.
+ *   active [S,B] uint8; cache_o_in [S,B,Hq,d] bf16 bits; cache_lse_in [S,B,Hq] double
+ *   o_out, cache_o_out [S,B,Hq,d] double; lse_out, cache_lse_out [S,B,Hq] double
+ */
+int oracle_sparse_losa(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                       const int32_t *page_table, const int32_t *n_ctx, const int32_t *idx,
+                       const int32_t *cnt, int kmax, const uint16_t *blk_k, const uint16_t *blk_v,
+                       const uint8_t *active, const uint16_t *cache_o_in, const double *cache_lse_in,
+                       int S, int B, int Hq, int Hkv, int d, int P, int max_pages, long n_phys,
+                       double *o_out, double *lse_out, double *cache_o_out, double *cache_lse_out) {
+  if (check_dims(S, B, Hq, Hkv, d, P, max_pages) != ORACLE_OK || kmax <= 0)
+    return ORACLE_EINVAL;
+  for (int s = 0; s < S; ++s) {
+    if (n_ctx[s] <= 0 || n_ctx[s] > max_pages * P) return ORACLE_EINVAL;
+    const int np = (n_ctx[s] + P - 1) / P;
+    for (int h = 0; h < Hkv; ++h) {
+      const int32_t *row = idx + ((size_t)s * Hkv + h) * kmax;
+      const int c0 = cnt[(size_t)s * Hkv + h];
+      if (c0 < 0 || c0 > kmax) return ORACLE_EINDEX;
+      for (int r = 0; r < c0; ++r) {
+        if (row[r] < 0 || row[r] >= np) return ORACLE_EINDEX;
+        for (int r2 = 0; r2 < r; ++r2)
+          if (row[r2] == row[r]) return ORACLE_EINDEX;
+        if (phys_page(page_table, s, row[r], max_pages, n_phys) < 0) return ORACLE_EPAGE;
+      }
+    }
+  }
+  const int G = Hq / Hkv;
+  const double c = 1.0 / sqrt((double)d);
+  int status = ORACLE_OK;
+
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int sh = 0; sh < S * Hkv; ++sh) {
+    const int s = sh / Hkv, h = sh % Hkv;
+    const int n = n_ctx[s];
+    const int32_t *sel = idx + (size_t)sh * kmax;
+    const int nsel = cnt[sh];
+    const int npre_max = nsel * P;
+    const uint16_t **krow = (const uint16_t **)malloc(sizeof(void *) * (size_t)(npre_max + 1));
+    const uint16_t **vrow = (const uint16_t **)malloc(sizeof(void *) * (size_t)(npre_max + 1));
+    double *logit = (double *)malloc(sizeof(double) * (size_t)(npre_max + B + 1));
+    double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+    double *op = (double *)malloc(sizeof(double) * (size_t)d);
+    double *ob = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!krow || !vrow || !logit || !qd || !op || !ob) {
+#pragma omp atomic write
+      status = ORACLE_ENOMEM;
+      free(krow); free(vrow); free(logit); free(qd); free(op); free(ob);
+      continue;
+    }
+    /* the prefix key set: valid tokens of the selected pages */
+    int npre = 0;
+    for (int r = 0; r < nsel; ++r) {
+      const int lp = sel[r];
+      const long pp = phys_page(page_table, s, lp, max_pages, n_phys);
+      for (int slot = 0; slot < P && lp * P + slot < n; ++slot) {
+        krow[npre] = cache_row(k, pp, h, slot, Hkv, P, d);
+        vrow[npre] = cache_row(v, pp, h, slot, Hkv, P, d);
+        ++npre;
+      }
+    }
+    for (int b = 0; b < B; ++b) {
+      const int act = active[(size_t)s * B + b] != 0;
+      for (int g = 0; g < G; ++g) {
+        const int j = h * G + g;
+        const size_t ro = ((size_t)s * B + b) * Hq + j;
+        const size_t qoff = ro * (size_t)d;
+        for (int i = 0; i < d; ++i) qd[i] = widen_bf16(q[qoff + i]);
+        /* prefix part: computed for an active token, from the cache otherwise */
+        double lse_p;
+        if (act) {
+          double mx = -INFINITY;
+          for (int t = 0; t < npre; ++t) {
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i) dot += qd[i] * widen_bf16(krow[t][i]);
+            logit[t] = c * dot;
+            if (logit[t] > mx) mx = logit[t];
+          }
+          for (int i = 0; i < d; ++i) op[i] = 0.0;
+          if (npre > 0) {
+            double sum = 0.0;
+            for (int t = 0; t < npre; ++t) sum += exp(logit[t] - mx);
+            for (int t = 0; t < npre; ++t) {
+              const double p = exp(logit[t] - mx) / sum;
+              for (int i = 0; i < d; ++i) op[i] += p * widen_bf16(vrow[t][i]);
+            }
+            lse_p = mx + log(sum);
+          } else {
+            lse_p = -INFINITY;
+          }
+        } else {
+          for (int i = 0; i < d; ++i) op[i] = widen_bf16(cache_o_in[qoff + i]);
+          lse_p = cache_lse_in[ro];
+        }
+        for (int i = 0; i < d; ++i) cache_o_out[qoff + i] = op[i];
+        cache_lse_out[ro] = lse_p;
+        /* block part: the block's own B tokens, no mask */
+        double mx = -INFINITY;
+        for (int u = 0; u < B; ++u) {
+          const size_t off = (((size_t)s * B + u) * Hkv + h) * (size_t)d;
+          double dot = 0.0;
+          for (int i = 0; i < d; ++i) dot += qd[i] * widen_bf16(blk_k[off + i]);
+          logit[u] = c * dot;
+          if (logit[u] > mx) mx = logit[u];
+        }
+        double sum = 0.0;
+        for (int u = 0; u < B; ++u) sum += exp(logit[u] - mx);
+        for (int i = 0; i < d; ++i) ob[i] = 0.0;
+        for (int u = 0; u < B; ++u) {
+          const size_t off = (((size_t)s * B + u) * Hkv + h) * (size_t)d;
+          const double p = exp(logit[u] - mx) / sum;
+          for (int i = 0; i < d; ++i) ob[i] += p * widen_bf16(blk_v[off + i]);
+        }
+        const double lse_b = mx + log(sum);
+        /* merge of the two parts */
+        const double top = lse_p > lse_b ? lse_p : lse_b;
+        const double wp = lse_p == -INFINITY ? 0.0 : exp(lse_p - top);
+        const double wb = exp(lse_b - top);
+        const double lse = top + log(wp + wb);
+        for (int i = 0; i < d; ++i) o_out[qoff + i] = (wp * op[i] + wb * ob[i]) / (wp + wb);
+        lse_out[ro] = lse;
+      }
+    }
+    free(krow); free(vrow); free(logit); free(qd); free(op); free(ob);
+  }
+  return status;
+}

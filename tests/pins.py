@@ -417,10 +417,74 @@ def pin_global_concentrated_head(orc):
     assert r.cnt[0, 1] == w.Hkv * w.kmax - len(pages)
 
 
+# ---------------------------------------------------------- LoSA prefix reuse
+def run_losa(orc, w, idx, cnt, active, cache_o, cache_lse, q=None, bk=None, bv=None):
+    return orc.sparse_losa(W.bits(w.q1 if q is None else q), W.bits(w.k_cache), W.bits(w.v_cache),
+                           w.n_ctx.numpy(), idx, cnt, W.bits(w.blk_k1 if bk is None else bk),
+                           W.bits(w.blk_v1 if bv is None else bv), active, cache_o, cache_lse,
+                           page_table=None if w.page_table is None else w.page_table.numpy(),
+                           max_pages=w.max_pages)
+
+
+def selected_kv(w, s, h, pages):
+    """K, V [n_sel, d] float64 of the valid tokens of the given logical pages."""
+    n = int(w.n_ctx[s])
+    kc, vc = f64(w.k_cache), f64(w.v_cache)
+    Ks, Vs = [], []
+    for lp in pages:
+        pp = w.physical_page(s, int(lp))
+        valid = min(w.P, n - int(lp) * w.P)
+        Ks.append(kc[pp, h, :valid])
+        Vs.append(vc[pp, h, :valid])
+    return (np.concatenate(Ks, axis=0), np.concatenate(Vs, axis=0)) if Ks else (None, None)
+
+
+def pin_losa(orc):
+    """Reuse of the prefix part (LoSA): with a mixed active mask, an active row's prefix
+    part (written to the new cache) is softmax attention over the selected pages, and
+    every row's output is the log-sum-exp merge of its prefix part (fresh, or the cache's
+    for a stable row) with softmax attention over the block, all written with numpy; with
+    every token active the output is the plain sparse pass."""
+    w = small_paged(4)
+    r = run(orc, w)
+    rng = np.random.default_rng(5)
+    active = rng.random((w.S, w.B)) < 0.5
+    active[0, 0], active[0, 1] = True, False
+    cache_o = W.bits(torch.randn(w.q1.shape, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16))
+    cache_lse = rng.normal(0.0, 2.0, (w.S, w.B, w.Hq))
+    o, lse, co, cl = run_losa(orc, w, r.idx, r.cnt, active, cache_o, cache_lse)
+    q, bk, bv, cof = f64(w.q1), f64(w.blk_k1), f64(w.blk_v1), f64(cache_o)
+    c = 1.0 / math.sqrt(w.d)
+    for s in range(w.S):
+        for h in range(w.Hkv):
+            Kp, Vp = selected_kv(w, s, h, r.idx[s, h, :r.cnt[s, h]])
+            Qh = group_queries(q, s, h, w.G)                       # rows (b, g) in order
+            op_f, lp_f = attention_np(Qh, Kp, Vp, c)
+            ob, lb = attention_np(Qh, bk[s, :, h], bv[s, :, h], c)
+            for b in range(w.B):
+                for g in range(w.G):
+                    row, j = b * w.G + g, h * w.G + g
+                    if active[s, b]:
+                        op, lp = op_f[row], lp_f[row]
+                        assert np.max(np.abs(co[s, b, j] - op)) < 1e-12 and abs(cl[s, b, j] - lp) < 1e-12
+                    else:
+                        op, lp = cof[s, b, j], cache_lse[s, b, j]
+                        assert np.array_equal(co[s, b, j], op) and cl[s, b, j] == lp
+                    top = max(lp, lb[row])
+                    wp, wb = math.exp(lp - top), math.exp(lb[row] - top)
+                    ref = (wp * op + wb * ob[row]) / (wp + wb)
+                    assert np.max(np.abs(o[s, b, j] - ref)) < 1e-12, (s, h, b, g)
+                    assert abs(lse[s, b, j] - (top + math.log(wp + wb))) < 1e-12
+    # every token active: the plain sparse pass
+    o2, lse2, _, _ = run_losa(orc, w, r.idx, r.cnt, np.ones((w.S, w.B), bool), cache_o, cache_lse)
+    ref_o, ref_lse = run_sparse(orc, w, r.idx, r.cnt)
+    assert np.max(np.abs(o2 - ref_o)) < 1e-12 and np.max(np.abs(lse2 - ref_lse)) < 1e-12
+
+
 FAST_PINS = [pin_score_sums, pin_dense_equivalence, pin_topk_brute_force,
              pin_exact_tie_lower_index, pin_planted_needles, pin_merge_identity,
              pin_selection_output_is_prefix_attention, pin_page_table_invariance,
              pin_query_order_invariance, pin_single_row, pin_budget_covers_prefix,
              pin_ascending_and_padding, pin_worked_example, pin_rejects_bad_indices,
              pin_global_brute_force, pin_global_one_head_is_per_head, pin_global_covers_prefix,
-             pin_global_concentrated_head]
+             pin_global_concentrated_head, pin_losa]

@@ -52,6 +52,10 @@ MUTANTS = [
      "const long budget = (long)(topk[s] / P);", 0),
     ("global_items_head_ignored", "items[h * np + lp].score = score[((size_t)s * Hkv + h) * max_pages + lp];",
      "items[h * np + lp].score = score[((size_t)s * Hkv + 0) * max_pages + lp];", 0),
+    ("losa_cache_for_active", "const int act = active[(size_t)s * B + b] != 0;",
+     "const int act = active[(size_t)s * B + b] == 0;", 0),
+    ("losa_block_dropped", "const double wb = exp(lse_b - top);", "const double wb = 0.0 * exp(lse_b - top);", 0),
+    ("losa_cache_lse_ignored", "lse_p = cache_lse_in[ro];", "lse_p = 0.0;", 0),
     ("global_pages_unsorted", "qsort(chosen, (size_t)take, sizeof(int), by_int); /* head-major",
      "(void)by_int; /* head-major", 0),
 ]
