@@ -452,7 +452,20 @@ def _run_ours(args, world, rank, local, dsa):
     hb_sp_us = 1e3 * timed(lambda i: dwh.sparse(dwh.q1, dwh.blk_k1, dwh.blk_v1), 50, cur)
     ph_sp_us = 1e3 * timed(lambda i: dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1), 50, cur)
     hb_cnt = dwh.cnt.cpu().numpy()
-    del dw, dwh, qs
+    # prefix-part reuse (LoSA): a sparse step whose tokens are all stable reads its
+    # prefix parts from the caches and loads no page; one with every token active
+    # computes them and refreshes the caches
+    c_o = torch.empty_like(dw.q1)
+    c_l = torch.empty(w.q1.shape[:3], dtype=torch.float32, device="cuda")
+    on = torch.ones((w.S, w.B), dtype=torch.uint8, device="cuda")
+    off = torch.zeros_like(on)
+    for i in range(3):
+        dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1, active=on, cache=(c_o, c_l))
+    losa_active_us = 1e3 * timed(lambda i: dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1, active=on,
+                                                       cache=(c_o, c_l)), 50, cur)
+    losa_stable_us = 1e3 * timed(lambda i: dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1, active=off,
+                                                       cache=(c_o, c_l)), 50, cur)
+    del dw, dwh, qs, c_o, c_l
 
     if rank != 0:
         return
@@ -507,6 +520,11 @@ def _run_ours(args, world, rank, local, dsa):
                         "per_head_sparse_step_us": round(ph_sp_us, 2),
                         "pages_per_head_min": int(hb_cnt.min()),
                         "pages_per_head_max": int(hb_cnt.max())},
+        "prefix_reuse": {"what": "sparse step with the prefix part of stable tokens reused from "
+                                 "caches (dsa_dims.active); eager launches",
+                         "all_active_us": round(losa_active_us, 2),
+                         "all_stable_us": round(losa_stable_us, 2),
+                         "per_head_sparse_step_us": round(ph_sp_us, 2)},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)

@@ -60,6 +60,9 @@ int make_shape(const dsa_dims *dims, Shape *out) {
   s.sm_limit = d.sm_limit;
   s.lse_out = d.lse_out;
   s.head_budget = d.head_budget;
+  s.active = d.active;
+  s.prefix_o = static_cast<__nv_bfloat16 *>(d.prefix_o_cache);
+  s.prefix_lse = d.prefix_lse_cache;
   *out = s;
   return DSA_OK;
 }
@@ -282,6 +285,9 @@ int dsa_sparse_attn(const void *q_blk, const void *k_cache, const void *v_cache,
     return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(blk_k) ||
       !aligned16(blk_v) || !aligned16(o_out) || !aligned16(workspace))
+    return DSA_ERR_INVALID_ARG;
+  if (sh.active && (!sh.prefix_o || !sh.prefix_lse || !aligned16(sh.prefix_o) ||
+                    (reinterpret_cast<uintptr_t>(sh.prefix_lse) & 3u) != 0))
     return DSA_ERR_INVALID_ARG;
   const dsa::SparsePlan plan = dsa::plan_sparse(sh, num_sms_current());
   if (ws_bytes < plan.total) return DSA_ERR_WORKSPACE_TOO_SMALL;

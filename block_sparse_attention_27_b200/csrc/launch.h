@@ -18,6 +18,9 @@ struct Shape {
   int sm_limit;               // selection pass: SMs it may hold (0 = all)
   float *lse_out;             // optional [S, B, Hq]: each row's log-sum-exp (natural log)
   int head_budget;            // selection pass: 1 = one budget of Hkv*kp pages per sequence
+  const uint8_t *active;      // sparse pass: optional [S, B] active tokens (prefix-part reuse)
+  __nv_bfloat16 *prefix_o;    // with active: [S, B, Hq, D] normalised prefix parts
+  float *prefix_lse;          // with active: [S, B, Hq] their log-sum-exps (natural log)
 };
 
 // TMA map of a paged cache [n_phys, Hkv, P, D] viewed as rows of D bf16; boxes of

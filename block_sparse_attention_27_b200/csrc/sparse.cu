@@ -278,6 +278,15 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     if (reporter) raise_status(a.status, kStatusBadIndex);
     cnt = max(0, min(cnt, sh.kmax));
   }
+  if (sh.active && !blk_cta) {
+    // prefix-part reuse: a row tile whose tokens are all stable needs no page
+    // (each warp checks the tile's tokens itself: a warp-uniform answer)
+    const int lane = threadIdx.x & 31;
+    const int b0 = row_base / sh.G, b1 = min(sh.B, (row_base + kRowsPerCta + sh.G - 1) / sh.G);
+    bool any = false;
+    for (int b = b0 + lane; b < b1; b += 32) any |= sh.active[(size_t)s * sh.B + b] != 0;
+    if (!__any_sync(0xffffffffu, any)) cnt = 0;
+  }
   if (threadIdx.x == 0) DSA_TRACE_AFTER(34, cnt + n);
   // the page CTAs split this head's cnt pages evenly, in whole tiles (counts
   // differ per head under the head-adaptive budget); ppc_eff = plan.ppc when
@@ -393,6 +402,89 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         v[j] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
+    const int grow = row_base + row;
+    const int b = grow / sh.G, g = grow % sh.G;
+    const size_t orow = ((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g;
+    if (sh.active) {
+      // prefix-part reuse: the page contributions (all but the last) merge into
+      // the prefix part; an active token keeps it and writes it to the cache, a
+      // stable one takes the cache's instead; then prefix and block part merge
+      float mp = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kMaxCluster - 1; ++j)
+        if (j < C - 1 && st[j].y > 0.f) mp = fmaxf(mp, st[j].x);
+      float lp = 0.f;
+      float op[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < kMaxCluster - 1; ++j) {
+        if (j >= C - 1 || !(st[j].y > 0.f)) continue;
+        const float w = exp2f(st[j].x - mp) * st[j].y;
+        lp += w;
+        const __half2 *hv = reinterpret_cast<const __half2 *>(&v[j]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hv[e]);
+          op[2 * e] = fmaf(w, f.x, op[2 * e]);
+          op[2 * e + 1] = fmaf(w, f.y, op[2 * e + 1]);
+        }
+      }
+      float m1;  // prefix part: log2-domain log-sum-exp (-inf: empty), values normalised
+      __nv_bfloat16 *co = sh.prefix_o + orow * D + ch * 8;
+      if (sh.active[(size_t)s * sh.B + b] != 0) {
+        const float inv = lp > 0.f ? 1.f / lp : 0.f;
+        m1 = lp > 0.f ? mp + log2f(lp) : -INFINITY;
+        uint4 cv;
+        uint32_t *pc = reinterpret_cast<uint32_t *>(&cv);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          op[2 * e] *= inv;
+          op[2 * e + 1] *= inv;
+          __nv_bfloat162 bv = __floats2bfloat162_rn(op[2 * e], op[2 * e + 1]);
+          pc[e] = *reinterpret_cast<uint32_t *>(&bv);
+        }
+        *reinterpret_cast<uint4 *>(co) = cv;
+        if (ch == 0) sh.prefix_lse[orow] = m1 * 0.6931471805599453f;
+      } else {
+        const float lse_c = sh.prefix_lse[orow];
+        m1 = lse_c * 1.4426950408889634f;  // (-inf stays -inf)
+        const uint4 cv = *reinterpret_cast<const uint4 *>(co);
+        const __nv_bfloat162 *pc = reinterpret_cast<const __nv_bfloat162 *>(&cv);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(pc[e]);
+          op[2 * e] = f.x;
+          op[2 * e + 1] = f.y;
+        }
+      }
+      // the block part: the last contribution
+      float2 sb = make_float2(-INFINITY, 0.f);
+      uint4 vb = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int j = 0; j < kMaxCluster; ++j)
+        if (j == C - 1) {
+          sb = st[j];
+          vb = v[j];
+        }
+      const bool has_p = m1 > -INFINITY, has_b = sb.y > 0.f;
+      const float mm = fmaxf(has_p ? m1 : -INFINITY, has_b ? sb.x : -INFINITY);
+      const float wp = has_p ? exp2f(m1 - mm) : 0.f;
+      const float wb = has_b ? exp2f(sb.x - mm) * sb.y : 0.f;
+      const float tot = wp + wb;
+      const float inv = tot > 0.f ? 1.f / tot : 0.f;
+      if (sh.lse_out && ch == 0) sh.lse_out[orow] = tot > 0.f ? (mm + log2f(tot)) * 0.6931471805599453f : -INFINITY;
+      const __half2 *hb = reinterpret_cast<const __half2 *>(&vb);
+      uint4 outv;
+      uint32_t *po = reinterpret_cast<uint32_t *>(&outv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(hb[e]);
+        __nv_bfloat162 bv = __floats2bfloat162_rn((wp * op[2 * e] + wb * f.x) * inv,
+                                                  (wp * op[2 * e + 1] + wb * f.y) * inv);
+        po[e] = *reinterpret_cast<uint32_t *>(&bv);
+      }
+      *reinterpret_cast<uint4 *>(a.o_out + orow * D + ch * 8) = outv;
+      continue;
+    }
     float mx = -INFINITY;
 #pragma unroll
     for (int j = 0; j < kMaxCluster; ++j)
@@ -413,8 +505,6 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       }
     }
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    const int grow = row_base + row;
-    const int b = grow / sh.G, g = grow % sh.G;
     if (sh.lse_out && ch == 0)  // the row's log-sum-exp over its key set: (M + log2 L) ln 2
       sh.lse_out[((size_t)s * sh.B + b) * sh.Hq + (size_t)h * sh.G + g] =
           lsum > 0.f ? (mx + log2f(lsum)) * 0.6931471805599453f : -INFINITY;

@@ -48,7 +48,8 @@ class dsa_dims(ctypes.Structure):
                 ("max_pages", ctypes.c_int32), ("kmax", ctypes.c_int32),
                 ("n_phys", ctypes.c_int64), ("page_table", ctypes.c_void_p),
                 ("sm_limit", ctypes.c_int32), ("lse_out", ctypes.c_void_p),
-                ("head_budget", ctypes.c_int32)]
+                ("head_budget", ctypes.c_int32), ("active", ctypes.c_void_p),
+                ("prefix_o_cache", ctypes.c_void_p), ("prefix_lse_cache", ctypes.c_void_p)]
 
 
 _lib = None
@@ -125,7 +126,7 @@ def make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table=None,
               sm_limit=0, head_budget=0) -> dsa_dims:
     return dsa_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys,
                     None if page_table is None else page_table.data_ptr(), int(sm_limit), None,
-                    int(head_budget))
+                    int(head_budget), None, None, None)
 
 
 def _with_lse(dims: dsa_dims, lse_out) -> dsa_dims:
@@ -228,8 +229,11 @@ def status_word(status, stream=None) -> int:
 
 
 def dsa_sparse_attn(q_blk, k_cache, v_cache, idx, blk_k, blk_v, o_out, stream=None, *,
-                    dims: dsa_dims, n_ctx, idx_cnt, workspace: Workspace, lse_out=None):
-    """Sparse pass (see include/dsa.h).  All tensors on the GPU; raises DsaError."""
+                    dims: dsa_dims, n_ctx, idx_cnt, workspace: Workspace, lse_out=None,
+                    active=None, prefix_o_cache=None, prefix_lse_cache=None):
+    """Sparse pass (see include/dsa.h).  All tensors on the GPU; raises DsaError.
+    active (uint8 [S, B]) with prefix_o_cache (bf16 [S, B, Hq, d]) and prefix_lse_cache
+    (fp32 [S, B, Hq]): reuse of the prefix part for stable tokens."""
     _check(q_blk, "q_blk", torch.bfloat16, 4)
     _check(k_cache, "k_cache", torch.bfloat16, 4)
     _check(v_cache, "v_cache", torch.bfloat16, 4)
@@ -240,6 +244,14 @@ def dsa_sparse_attn(q_blk, k_cache, v_cache, idx, blk_k, blk_v, o_out, stream=No
     _check(n_ctx, "n_ctx", torch.int32)
     _check(idx_cnt, "idx_cnt", torch.int32)
     dims = _with_lse(dims, lse_out)
+    if active is not None:
+        _check(active, "active", torch.uint8)
+        _check(prefix_o_cache, "prefix_o_cache", torch.bfloat16)
+        _check(prefix_lse_cache, "prefix_lse_cache", torch.float32)
+        dims = dsa_dims.from_buffer_copy(dims)
+        dims.active = active.data_ptr()
+        dims.prefix_o_cache = prefix_o_cache.data_ptr()
+        dims.prefix_lse_cache = prefix_lse_cache.data_ptr()
     rc = load().dsa_sparse_attn(_ptr(q_blk), _ptr(k_cache), _ptr(v_cache), _ptr(idx), _ptr(blk_k),
                                 _ptr(blk_v), _ptr(o_out), _stream(stream), ctypes.byref(dims),
                                 _ptr(n_ctx), _ptr(idx_cnt), _ptr(workspace.buf), workspace.nbytes)
@@ -300,10 +312,14 @@ class DeviceWorkload:
                    cnt_out=self.cnt, workspace=self.ws_sel, lse_out=lse_out)
         return self.idx, self.cnt, self.o_sel
 
-    def sparse(self, q, blk_k, blk_v, idx=None, cnt=None, stream=None, out=None, lse_out=None):
+    def sparse(self, q, blk_k, blk_v, idx=None, cnt=None, stream=None, out=None, lse_out=None,
+               active=None, cache=None):
+        """cache = (prefix_o_cache, prefix_lse_cache), used with `active`."""
         o = self.o_sp if out is None else out
         dsa_sparse_attn(q, self.k_cache, self.v_cache, self.idx if idx is None else idx, blk_k,
                         blk_v, o, stream, dims=self.dims, n_ctx=self.n_ctx,
                         idx_cnt=self.cnt if cnt is None else cnt, workspace=self.ws_sp,
-                        lse_out=lse_out)
+                        lse_out=lse_out, active=active,
+                        prefix_o_cache=None if cache is None else cache[0],
+                        prefix_lse_cache=None if cache is None else cache[1])
         return o

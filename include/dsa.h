@@ -106,6 +106,20 @@ typedef struct dsa_dims {
                          holds a different count per head (cnt_out); kmax must hold every
                          head's count (min(max_pages, Hkv*kp) always does), else the call
                          reports DSA_ERR_BAD_INDEX and keeps that head's first kmax pages. */
+  const uint8_t *active; /* sparse pass: optional device [S, B], NULL = every token active.
+                         Reuse of the prefix part for stable tokens (LoSA page, abstract): a
+                         row (b, query head) splits its attention into the prefix part (the
+                         selected pages) and the block part (the block's B tokens).  For
+                         active[s,b] != 0 the prefix part is computed and written to the two
+                         caches below; for a stable token (0) it is read from them.  The block
+                         part is always computed and the row's output is the log-sum-exp
+                         merge of the two parts.  A (sequence, KV head, 128-row tile) whose
+                         tokens are all stable loads no page at all. */
+  void *prefix_o_cache;  /* with active: device bf16 [S, B, Hq, d], 16-byte aligned: each row's
+                         normalised prefix part (softmax over the selected pages times V) */
+  float *prefix_lse_cache; /* with active: device fp32 [S, B, Hq]: its log-sum-exp, natural log
+                         (-inf: no prefix key).  A stable row reads whatever its cache holds:
+                         fill the caches with a call whose tokens are all active first. */
 } dsa_dims;
 
 /* cudaStream_t without including the CUDA headers. */

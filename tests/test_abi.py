@@ -149,3 +149,17 @@ def test_select_launches(lib):
     assert dsa.select_launches(good_dims(S=100, Hq=28, Hkv=4)) == 6
     with pytest.raises(dsa.DsaError):
         dsa.select_launches(good_dims(d=96))
+
+
+def test_prefix_reuse_needs_both_caches(lib):
+    """dims.active without the two prefix caches (or with a misaligned one) is rejected
+    on the host, before anything is launched."""
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    for o_cache, lse_cache in ((None, None), (1 << 20, None), ((1 << 20) + 8, 1 << 20)):
+        dims = good_dims()
+        dims.active = 1 << 20
+        dims.prefix_o_cache = o_cache
+        dims.prefix_lse_cache = lse_cache
+        rc = lib.dsa_sparse_attn(fake, fake, fake, fake, fake, fake, fake, None, ctypes.byref(dims),
+                                 fake, fake, fake, 1 << 30)
+        assert rc == dsa.DSA_ERR_INVALID_ARG
