@@ -210,6 +210,45 @@ def oracle_block(w, steps):
     return time.perf_counter() - t0
 
 
+def block_time_shape(dsa, names=("8k", "32k", "128k"), reps=20):
+    """One layer of a denoising block at several context lengths, with a GEMM stand-in
+    for the FFN (two bf16 matmuls, d_model = Hq*d, d_ff = 4*d_model, S*B tokens, random
+    weights; cuBLAS through torch).  Per context: the selection pass (exact attention of
+    the block's queries over the prefix, the dense stand-in), the sparse step and the FFN
+    in microseconds (eager launches, CUDA events), attention's share of a block's time
+    and the block speed-up of shared-index sparse attention over exact attention at every
+    step: 32 x (exact + ffn) / (select + 31 x sparse + 32 x ffn)."""
+    out = {}
+    cur = torch.cuda.current_stream()
+    for name in names:
+        w = W.make(name, 0)
+        dw = dsa.DeviceWorkload(w)
+        dm = w.Hq * w.d
+        g = torch.Generator(device="cuda")
+        g.manual_seed(1)
+        x = torch.randn((w.S * w.B, dm), device="cuda", generator=g, dtype=torch.float32).to(torch.bfloat16)
+        w1 = (torch.randn((dm, 4 * dm), device="cuda", generator=g, dtype=torch.float32) / dm ** 0.5).to(torch.bfloat16)
+        w2 = (torch.randn((4 * dm, dm), device="cuda", generator=g, dtype=torch.float32) / (4 * dm) ** 0.5).to(torch.bfloat16)
+        ffn = lambda i: torch.matmul(torch.matmul(x, w1), w2)  # noqa: E731
+        for i in range(3):
+            dw.select()
+            dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1)
+            ffn(i)
+        sel_us = 1e3 * timed(lambda i: dw.select(), reps, cur)
+        sp_us = 1e3 * timed(lambda i: dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1), reps, cur)
+        ffn_us = 1e3 * timed(ffn, reps, cur)
+        T = w.T
+        sparse_block = sel_us + (T - 1) * sp_us + T * ffn_us
+        dense_block = T * (sel_us + ffn_us)
+        out[name] = {"select_us": round(sel_us, 1), "sparse_step_us": round(sp_us, 2),
+                     "ffn_us": round(ffn_us, 2),
+                     "attention_share_sparse": round((sel_us + (T - 1) * sp_us) / sparse_block, 3),
+                     "attention_share_exact": round(T * sel_us / dense_block, 3),
+                     "block_speedup": round(dense_block / sparse_block, 2)}
+        del dw, x, w1, w2
+    return out
+
+
 def cpu_baseline(w):
     import oracle
     steps = w.T - 1
@@ -466,6 +505,7 @@ def _run_ours(args, world, rank, local, dsa):
     losa_stable_us = 1e3 * timed(lambda i: dw.sparse(dw.q1, dw.blk_k1, dw.blk_v1, active=off,
                                                        cache=(c_o, c_l)), 50, cur)
     del dw, dwh, qs, c_o, c_l
+    shape = block_time_shape(dsa)
 
     if rank != 0:
         return
@@ -525,6 +565,11 @@ def _run_ours(args, world, rank, local, dsa):
                          "all_active_us": round(losa_active_us, 2),
                          "all_stable_us": round(losa_stable_us, 2),
                          "per_head_sparse_step_us": round(ph_sp_us, 2)},
+        "block_time_shape": {"what": "one layer, GEMM stand-in for the FFN (d_ff = 4 d_model, "
+                                     "random bf16 weights, cuBLAS): selection pass as exact "
+                                     "attention, attention share of a block and block speed-up "
+                                     "of sparse over exact attention at every step; eager launches",
+                             **shape},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
