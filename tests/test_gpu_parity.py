@@ -199,3 +199,38 @@ def test_repeatable_on_poisoned_workspaces(dsa_mod):
         else:
             for a, b in zip(first, got):
                 assert torch.equal(a, b)
+
+
+def test_empty_prefix(dsa_mod):
+    """A sequence with an empty prefix (n_ctx = 0) beside a normal one: its selection
+    keeps no page (idx -1, cnt 0, o_out 0, log-sum-exp -inf), its sparse step attends
+    to the block alone (numpy softmax over the block), and the other sequence's results
+    are bit for bit those of a run where the first sequence has its prefix."""
+    w = W.make("batched", 0, S=2, n_lo=500, n_hi=1500, B=8, Hq=8, Hkv=2, topk_choices=(64,))
+    base = dsa_mod.DeviceWorkload(w)
+    base.select()
+    q, bk, bv = (x.cuda() for x in w.step_inputs(2))
+    o_base = base.sparse(q, bk, bv).clone()
+    w.n_ctx[0] = 0
+    dw = dsa_mod.DeviceWorkload(w)
+    lse = torch.empty(w.q1.shape[:3], dtype=torch.float32, device="cuda")
+    dw.select(lse_out=lse)
+    o = dw.sparse(q, bk, bv)
+    torch.cuda.synchronize()
+    assert dw.ws_sel.status() == dsa_mod.DSA_OK and dw.ws_sp.status() == dsa_mod.DSA_OK
+    assert int(dw.cnt[0].abs().sum()) == 0 and bool((dw.idx[0] == -1).all())
+    assert bool((dw.o_sel[0] == 0).all()) and bool(torch.isneginf(lse[0]).all())
+    # the block alone
+    qf, kf, vf = (x.double().cpu().numpy() for x in (w.step_inputs(2)[0][0], w.step_inputs(2)[1][0],
+                                                     w.step_inputs(2)[2][0]))
+    c = 1.0 / np.sqrt(w.d)
+    for j in range(w.Hq):
+        h = j // w.G
+        x = c * qf[:, j] @ kf[:, h].T
+        p = np.exp(x - x.max(axis=1, keepdims=True))
+        ref = (p / p.sum(axis=1, keepdims=True)) @ vf[:, h]
+        got = o[0, :, j].double().cpu().numpy()
+        assert np.max(np.abs(got - ref)) <= parity.MAX_ABS
+    # the other sequence is untouched
+    assert torch.equal(dw.idx[1], base.idx[1]) and torch.equal(dw.o_sel[1], base.o_sel[1])
+    assert torch.equal(o[1], o_base[1])
