@@ -147,6 +147,9 @@ def test_select_launches(lib):
     assert dsa.select_launches(good_dims(S=64)) == 4
     # 224 query rows per KV head: two 128-row tiles per group, 74 groups per launch
     assert dsa.select_launches(good_dims(S=100, Hq=28, Hkv=4)) == 6
+    # the head-adaptive budget adds its per-sequence selection kernel
+    assert dsa.select_launches(good_dims(head_budget=1)) == 2
+    assert dsa.select_launches(good_dims(S=64, head_budget=1)) == 5
     with pytest.raises(dsa.DsaError):
         dsa.select_launches(good_dims(d=96))
 
