@@ -23,6 +23,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -84,11 +85,17 @@ def load_peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of the kernel sources with comments and blank lines removed: editing a
+    comment keeps the recorded traffic, any change to the code drops it."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_attention_27_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+        h.update(name.encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 

@@ -3,25 +3,25 @@
 // KV head ("MAGE: All-[MASK] Block Already Knows Where to Look in Block
 // Diffusion LLM", Approach).
 //
-// One kernel, select_fused, launched cooperatively (all its CTAs co-resident).
-// A group is one (sequence, KV head); its CTAs are the (split, 128-row tile)
-// pairs, one wave over the SMs.
-//   1. Split-KV attention on the tcgen05 engine (tc_attn.cuh): the split's
-//      64-token tiles stream through a TMA ring.  Per split the CTA writes the
-//      unnormalised output O_j with its row max m_j and sum l_j, and per (tile,
-//      row) the partial probability mass of each unit of the tile (min(page, 32)
-//      keys of one page) relative to the row's reference max at that tile
-//      (pagepart, [tile][row][unit]), together with that max (mtile).
+// select_fused, launched cooperatively (all its CTAs co-resident).  A group is
+// one (sequence, KV head); its CTAs are the (split, 128-row tile) pairs.
+//   1. Split-KV attention on the tcgen05 engine (tc_attn.cuh).  Per split: the
+//      unnormalised O_j with row max m_j and sum l_j; per (tile, row): the mass
+//      of each unit of the tile (min(page, 32) keys of one page) relative to the
+//      row's reference max (pagepart), and that max (mtile).
 //   2. Group barrier: a counter in the workspace header, bounded wait.
-//   3. Every CTA of the group forms each row's global M = max_j m_j and
-//      L = sum_j l_j 2^(m_j - M), writes its share of the rows of o_out, and
-//      turns the partial masses of its share of the pages into page scores
-//        S_h[q] = (1/BG) sum_rows pagepart * 2^(mtile - M) / L,
-//      then keeps its local top-kp pages (radix select, ties to the lower page)
-//      as candidates, in ascending page order.
-//   4. The group's last CTA to finish step 3 selects the kp largest among the
-//      candidates (the global top-kp of the head is among them: each of its
-//      pages is in the local top-kp of its own CTA) and writes them ascending.
+//   3. Every CTA forms each row's M = max_j m_j and L = sum_j l_j 2^(m_j - M),
+//      scores the pages of its own tiles from partials bulk-copied into shared
+//      memory,  S_h[q] = (1/BG) sum_rows pagepart * 2^(mtile - M) / L,  and
+//      keeps its local top-kp as candidates (warp bitonic lists of (score,
+//      page) keys for kp <= 128, a radix select beyond).
+//   4. The group's last CTA to hand in its candidates selects the kp largest
+//      (the head's top-kp is among them: each of its pages is in the local
+//      top-kp of its own CTA) and writes them ascending.
+//   5. Every CTA merges rows of o_out = sum_j 2^(m_j - M) O_j / L, taken from
+//      a counter.
+// select_global_topk (head-adaptive budget only) then selects over all KV
+// heads of each sequence, from the page scores select_fused wrote.
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -190,7 +190,7 @@ struct SelectPolicy {
 };
 
 // ---------------------------------------------------------------------------
-// Steps 3-4 of the tail: the splits' row statistics, page scores, output rows.
+// Steps 3 and 5 of the tail: the splits' row statistics and the output rows.
 // ---------------------------------------------------------------------------
 // Folds a partial (m, l) into the running (M, L) of a row (log2 domain); an
 // empty partial (l = 0) leaves it unchanged.
