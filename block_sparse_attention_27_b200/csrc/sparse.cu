@@ -6,15 +6,18 @@
 //
 // One launch per step.  A thread-block cluster of C CTAs serves one (sequence,
 // KV head, 128-row tile): CTAs 0..C-2 run the tcgen05 engine (tc_attn.cuh) over
-// their slices [c*ppc, (c+1)*ppc) of the selected pages, gathered with TMA
-// through the page table; CTA C-1 takes the block's own tokens (a 3-D TMA box
-// over blk_k / blk_v), so that no CTA carries both.  The C partial results are
-// then merged: every softmax thread writes its row, normalised, in fp16 with
-// the row's (m, l), to this cluster's exchange area in the workspace (L2); after
-// one cluster barrier (release / acquire) the CTA that owns a row reads the C
-// contributions of its rows, combines them and writes o_out in bf16.  The
-// cluster only provides the co-scheduling and the barrier: going through L2
-// moves the partial rows faster than stores into the owners' shared memory.
+// even slices (whole tiles) of the head's own count of selected pages, gathered
+// with TMA through the page table; CTA C-1 takes the block's own tokens (a 3-D
+// TMA box over blk_k / blk_v).  The C partial results are then merged: every
+// softmax thread writes its row, normalised, in fp16 with the row's (m, l), to
+// this cluster's exchange area in the workspace (L2); after one cluster barrier
+// (release / acquire) the CTA that owns a row combines its C contributions and
+// writes o_out in bf16.  The cluster only provides the co-scheduling and the
+// barrier: going through L2 moves the partial rows faster than stores into the
+// owners' shared memory.  With dims.active (reuse of the prefix part of stable
+// tokens, "LoSA: Locality Aware Sparse Attention for Block-Wise Diffusion
+// Language Models", abstract) the page contributions form the prefix part, which
+// is taken from or written to the caches and then merged with the block part.
 #include <cuda_fp16.h>
 
 #include <algorithm>
