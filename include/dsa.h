@@ -206,8 +206,8 @@ int dsa_get_status(const void *workspace, dsa_stream_t stream);
  * DSA_SELECT_STATIC_SCRATCH_BYTES; a larger shape returns DSA_ERR_SCRATCH_LIMIT
  * before anything is launched (use dsa_select with a caller workspace).  On a
  * 148-SM B200 this admits an 8K prefix with 8 KV heads, 32 query tokens,
- * d = 128, page 16 (10.6 MiB) and a 32K prefix with 4 KV heads, page 64
- * (13.3 MiB), not a 128K prefix with 8 KV heads (49 MiB).
+ * d = 128, page 16 (10.7 MiB) and a 32K prefix with 4 KV heads, page 64
+ * (13.3 MiB), not a 128K prefix with 8 KV heads (49.5 MiB).
  *
  * Arguments: those of dsa_select without workspace/ws_bytes, plus
  *   status: device uint32, caller-owned, 4-byte aligned, receiving the device
