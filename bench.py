@@ -323,7 +323,10 @@ class Bench:
         self.n_ctx = w.n_ctx.to(dev)
         self.topk = w.topk.to(dev)
         self.page_table = None if w.page_table is None else w.page_table.to(dev)
-        self.dims = dsa.dims_for(self.q[0, 0], self.k[0], w.max_pages, w.kmax, self.page_table)
+        # the sparse steps reuse indices the selection wrote one block earlier (on the side
+        # stream, joined by an event): each gathers its pages before the kernel ahead of it ends
+        self.dims = dsa.dims_for(self.q[0, 0], self.k[0], w.max_pages, w.kmax, self.page_table,
+                                 early_gather=1)
         self.idx = torch.full((2, layers, S, w.Hkv, w.kmax), -1, dtype=torch.int32, device=dev)
         self.cnt = torch.zeros((2, layers, S, w.Hkv), dtype=torch.int32, device=dev)
         self.o_sel = torch.empty((layers, *w.q1.shape), dtype=torch.bfloat16, device=dev)

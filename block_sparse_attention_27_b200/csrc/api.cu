@@ -51,6 +51,7 @@ int make_shape(const dsa_dims *dims, Shape *out) {
   if (d.sm_limit < 0) return DSA_ERR_INVALID_ARG;
   if (d.head_budget != 0 && d.head_budget != 1) return DSA_ERR_INVALID_ARG;
   if (d.head_budget && d.Hkv > dsa::kMaxHeadsAdaptive) return DSA_ERR_UNSUPPORTED;
+  if (d.early_gather != 0 && d.early_gather != 1) return DSA_ERR_INVALID_ARG;
   Shape s{};
   s.S = d.S; s.B = d.B; s.Hq = d.Hq; s.Hkv = d.Hkv; s.G = G; s.BG = d.B * G;
   s.d = d.d; s.P = d.page; s.max_pages = d.max_pages; s.kmax = d.kmax;
@@ -63,6 +64,7 @@ int make_shape(const dsa_dims *dims, Shape *out) {
   s.active = d.active;
   s.prefix_o = static_cast<__nv_bfloat16 *>(d.prefix_o_cache);
   s.prefix_lse = d.prefix_lse_cache;
+  s.early_gather = (d.early_gather && !d.active) ? 1 : 0;  // prefix-part reuse decides per step
   *out = s;
   return DSA_OK;
 }
@@ -134,6 +136,14 @@ const char *dsa_strerror(int code) {
              "(use dsa_select with a caller workspace)";
     default: return "unknown status code";
   }
+}
+
+int dsa_sparse_kernel(const dsa_dims *dims) {
+  Shape sh;
+  const int rc = make_shape(dims, &sh);
+  if (rc != DSA_OK) return rc;
+  const int c = dsa::sparse_resident_cluster(sh);
+  return c > 0 ? 1 + c : 1;
 }
 
 int dsa_select_launches(const dsa_dims *dims) {

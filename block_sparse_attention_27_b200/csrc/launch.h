@@ -21,6 +21,7 @@ struct Shape {
   const uint8_t *active;      // sparse pass: optional [S, B] active tokens (prefix-part reuse)
   __nv_bfloat16 *prefix_o;    // with active: [S, B, Hq, D] normalised prefix parts
   float *prefix_lse;          // with active: [S, B, Hq] their log-sum-exps (natural log)
+  int early_gather;           // sparse pass: gather the selected pages before the dependency wait
 };
 
 // TMA map of a paged cache [n_phys, Hkv, P, D] viewed as rows of D bf16; boxes of
@@ -34,9 +35,14 @@ cudaError_t make_kv_pages_tensor_map(CUtensorMap *out, const void *base, long lo
                                      int P, int D, int pages);
 
 // The block's own keys/values [S*B, Hkv, D] bf16; boxes of 64 elements x 1 head x
-// 64 tokens with the 128-byte swizzle (tmap.cu).
+// box_tokens tokens with the 128-byte swizzle (tmap.cu).
 cudaError_t make_blk_tensor_map(CUtensorMap *out, const void *base, long long tokens, int Hkv,
-                                int D);
+                                int D, int box_tokens = 64);
+
+// The block's queries [S*B, Hq, D] bf16; boxes of 64 elements x G heads x
+// box_tokens tokens with the 128-byte swizzle (tmap.cu).
+cudaError_t make_q_tensor_map(CUtensorMap *out, const void *base, long long tokens, int Hq, int D,
+                              int G, int box_tokens);
 
 // Kernel launches issued by one dsa_select (when all its (sequence, KV head)
 // groups fit in one co-resident launch; see SelectPlan::launches) and by one
@@ -114,6 +120,13 @@ struct SparseArgs {
 };
 
 SparsePlan plan_sparse(const Shape &sh, int num_sms);
+// The sparse pass on the kernel whose CTAs hold all their keys in shared memory
+// (sparse_resident.cu): returns false (nothing launched) when the shape does not
+// fit it or uses prefix-part reuse; else launches and sets *err.
+bool launch_sparse_resident(const Shape &sh, const SparseArgs &a, cudaStream_t stream, cudaError_t *err);
+// Cluster size the all-keys-resident kernel would use for this shape on the
+// current device, 0 when the streaming kernel serves it.
+int sparse_resident_cluster(const Shape &sh);
 cudaError_t launch_sparse(const Shape &sh, const SparsePlan &plan, const SparseArgs &a,
                           cudaStream_t stream);
 

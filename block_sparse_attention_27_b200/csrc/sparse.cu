@@ -29,7 +29,6 @@
 namespace dsa {
 namespace {
 
-constexpr int kSpStages = 2;
 constexpr int kRowsPerCta = 128;
 constexpr int kMaxCluster = 16;
 
@@ -38,12 +37,12 @@ constexpr int kMaxCluster = 16;
 // the workspace: kMaxCluster slots (one per CTA), each the CTA's 128 partial rows
 // as [D/8 column chunks][128 rows][16 bytes] of fp16 (so a warp's stores of one
 // chunk are contiguous) followed by [128 rows] of (m, l) in fp32.
-template <int D>
+template <int D, int STG>
 struct SparseLayout {
   static constexpr uint32_t kSlotBytes = 128u * (2u * D + 8u);
   static __host__ __device__ constexpr uint32_t align16(uint32_t x) { return (x + 15u) & ~15u; }
   static __host__ __device__ constexpr uint32_t table_offset() {
-    return align16(tc::Layout<D, kSpStages>::kBytes);
+    return align16(tc::Layout<D, STG>::kBytes);
   }
   static __host__ __device__ constexpr uint32_t mask_offset(int ppc) {
     return table_offset() + 8u * (uint32_t)ppc;
@@ -190,13 +189,13 @@ struct SparsePolicy {
   __device__ __forceinline__ void after_tile(int, int, float, const float *) const {}
 };
 
-template <int D, int PAGE>
+template <int D, int PAGE, int STG>
 __global__ void __launch_bounds__(tc::kThreads, 1)
     sparse_attn(const __grid_constant__ SparseParams prm, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap kmap4,
                 const __grid_constant__ CUtensorMap vmap4, const __grid_constant__ CUtensorMap bkmap,
                 const __grid_constant__ CUtensorMap bvmap) {
-  using M = SparseLayout<D>;
+  using M = SparseLayout<D, STG>;
   extern __shared__ unsigned char smem_raw[];
   const Shape &sh = prm.sh;
   const SparsePlan &plan = prm.plan;
@@ -209,6 +208,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const int row_base = rt * kRowsPerCta;
   const bool blk_cta = c == C - 1;  // CTAs 0..C-2: pages; CTA C-1: the block's own tokens
   constexpr int kPagesPerTile = tc::kBN / PAGE;
+  const bool early = sh.early_gather != 0;
 
   SparsePolicy<D, PAGE> pol;
   pol.kmap = &kmap;
@@ -218,15 +218,92 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.bkmap = &bkmap;
   pol.bvmap = &bvmap;
   if (threadIdx.x == 0) DSA_TRACE_EVENT(0);
-  tc::Engine<D, kSpStages> eng;
+  tc::Engine<D, STG> eng;
   eng.setup(smem_raw, pol);
   if (threadIdx.x == 0) DSA_TRACE_EVENT(32);
+
+  const int32_t *idx_row = a.idx + sh_idx * sh.kmax;
+  pol.idx_row = idx_row;
+  pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
+  pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
+  pol.status = a.status;
+  pol.tab = nullptr;
+  pol.masks = nullptr;
+  pol.tab_off = M::table_offset();
+  pol.mask_off = M::mask_offset(plan.ppc);
+  pol.n_phys = sh.n_phys;
+  pol.phys0 = (long long)s * sh.max_pages;
+  pol.Hkv = sh.Hkv;
+  pol.h = h;
+  pol.G = sh.G;
+  pol.Hq = sh.Hq;
+  pol.B = sh.B;
+  pol.BG = sh.BG;
+  pol.s = s;
+  pol.row_base = row_base;
+  pol.sl2 = sh.sl2;
+
+  // The key side of the step: the prefix length, the count and (warp 0 of a page
+  // CTA) this CTA's slice of idx are loaded together (idx entries below kmax are
+  // always readable; the ones beyond the count are ignored), then this CTA's
+  // share of the pages.  With early gathering this runs before the dependency
+  // wait, else after it.
+  int num_tiles = 0;
+  auto key_side = [&]() {
+    const int n_raw = a.n_ctx[s];
+    int cnt = a.idx_cnt[sh_idx];
+    int lp_spec = -1;
+    if (threadIdx.x < 32 && !blk_cta) {
+      const int e = c * plan.ppc + (int)threadIdx.x;
+      if ((int)threadIdx.x < plan.ppc && e < sh.kmax) lp_spec = idx_row[e];
+    }
+    const bool reporter = threadIdx.x == 0 && c == 0 && rt == 0;
+    const int n = clamp_prefix(n_raw, sh.max_pages, PAGE, a.status, reporter && h == 0);
+    if (cnt < 0 || cnt > sh.kmax) {
+      if (reporter) raise_status(a.status, kStatusBadIndex);
+      cnt = max(0, min(cnt, sh.kmax));
+    }
+    if (sh.active && !blk_cta) {
+      // prefix-part reuse: a row tile whose tokens are all stable needs no page
+      // (each warp checks the tile's tokens itself: a warp-uniform answer)
+      const int lane = threadIdx.x & 31;
+      const int b0 = row_base / sh.G, b1 = min(sh.B, (row_base + kRowsPerCta + sh.G - 1) / sh.G);
+      bool any = false;
+      for (int b = b0 + lane; b < b1; b += 32) any |= sh.active[(size_t)s * sh.B + b] != 0;
+      if (!__any_sync(0xffffffffu, any)) cnt = 0;
+    }
+    if (threadIdx.x == 0) DSA_TRACE_AFTER(34, cnt + n);
+    // the page CTAs split this head's cnt pages evenly, in whole tiles (counts
+    // differ per head under the head-adaptive budget); ppc_eff = plan.ppc when
+    // cnt = kmax, and then the speculative idx load above is this CTA's slice
+    const int ppc_eff =
+        min(plan.ppc, ((cnt + C - 2) / (C - 1) + kPagesPerTile - 1) / kPagesPerTile * kPagesPerTile);
+    const int e_begin = blk_cta ? cnt : min(cnt, c * ppc_eff);
+    const int e_end = blk_cta ? cnt : min(cnt, (c + 1) * ppc_eff);
+    if (ppc_eff != plan.ppc) lp_spec = -2;  // not this slice's: prepare() loads it again
+    const int sel_tiles = (e_end - e_begin + kPagesPerTile - 1) / kPagesPerTile;
+    num_tiles = sel_tiles + (blk_cta ? plan.blk_tiles : 0);
+    pol.lp_spec = lp_spec;
+    pol.n = n;
+    pol.np = (n + PAGE - 1) / PAGE;
+    pol.e_begin = e_begin;
+    pol.e_end = e_end;
+    pol.sel_tiles = sel_tiles;
+  };
+
+  if (early) {
+    // everything the key side reads is, by the caller's contract, not written by
+    // the kernel ahead of this one: a page CTA builds its tables and has its
+    // first STG tiles in flight before the wait
+    key_side();
+    if (!blk_cta) eng.stage(pol, num_tiles);
+  }
   // While the kernel ahead of this one may still run: L2 prefetches of what this
-  // CTA will read.  The page list is read here without any ordering (through L2
-  // only, so that no stale line stays in L1) and serves only as prefetch
-  // addresses, clamped to the cache; everything the computation uses is read
-  // again after grid_dep_wait().  Warp 1 (the MMA issuer, idle until the first
-  // tiles land) and the softmax warps do this, not the producer.
+  // CTA will read.  Without early gathering the page list is read here without
+  // any ordering (through L2 only, so that no stale line stays in L1) and serves
+  // only as prefetch addresses, clamped to the cache; everything the computation
+  // uses is read again after grid_dep_wait().  Warp 1 (the MMA issuer, idle until
+  // the first tiles land) and the softmax warps do this, not the producer.
   if (eng.warp == 1) {
     const int lane = eng.lane;
     if (blk_cta) {
@@ -236,7 +313,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         sm100::prefetch_l2_bulk(bk + (size_t)u * sh.Hkv * D, D * 2);
         sm100::prefetch_l2_bulk(bv + (size_t)u * sh.Hkv * D, D * 2);
       }
-    } else {
+    } else if (!early) {
       const int e = c * plan.ppc + lane;
       if (lane < plan.ppc && e < sh.kmax) {
         const int lp = __ldcg(a.idx + sh_idx * sh.kmax + e);
@@ -263,70 +340,8 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   sm100::grid_dep_wait();
   sm100::grid_dep_launch_dependents();
   if (threadIdx.x == 0) DSA_TRACE_EVENT(33);
-
-  // the prefix length, the count and (warp 0 of a page CTA) this CTA's slice of
-  // idx are loaded together: idx entries below kmax are always readable, and
-  // the ones beyond the count are ignored
-  const int32_t *idx_row = a.idx + sh_idx * sh.kmax;
-  const int n_raw = a.n_ctx[s];
-  int cnt = a.idx_cnt[sh_idx];
-  int lp_spec = -1;
-  if (threadIdx.x < 32 && !blk_cta) {
-    const int e = c * plan.ppc + (int)threadIdx.x;
-    if ((int)threadIdx.x < plan.ppc && e < sh.kmax) lp_spec = idx_row[e];
-  }
-  const bool reporter = threadIdx.x == 0 && c == 0 && rt == 0;
-  const int n = clamp_prefix(n_raw, sh.max_pages, PAGE, a.status, reporter && h == 0);
-  if (cnt < 0 || cnt > sh.kmax) {
-    if (reporter) raise_status(a.status, kStatusBadIndex);
-    cnt = max(0, min(cnt, sh.kmax));
-  }
-  if (sh.active && !blk_cta) {
-    // prefix-part reuse: a row tile whose tokens are all stable needs no page
-    // (each warp checks the tile's tokens itself: a warp-uniform answer)
-    const int lane = threadIdx.x & 31;
-    const int b0 = row_base / sh.G, b1 = min(sh.B, (row_base + kRowsPerCta + sh.G - 1) / sh.G);
-    bool any = false;
-    for (int b = b0 + lane; b < b1; b += 32) any |= sh.active[(size_t)s * sh.B + b] != 0;
-    if (!__any_sync(0xffffffffu, any)) cnt = 0;
-  }
-  if (threadIdx.x == 0) DSA_TRACE_AFTER(34, cnt + n);
-  // the page CTAs split this head's cnt pages evenly, in whole tiles (counts
-  // differ per head under the head-adaptive budget); ppc_eff = plan.ppc when
-  // cnt = kmax, and then the speculative idx load above is this CTA's slice
-  const int ppc_eff = min(plan.ppc, ((cnt + C - 2) / (C - 1) + kPagesPerTile - 1) / kPagesPerTile * kPagesPerTile);
-  const int e_begin = blk_cta ? cnt : min(cnt, c * ppc_eff);
-  const int e_end = blk_cta ? cnt : min(cnt, (c + 1) * ppc_eff);
-  if (ppc_eff != plan.ppc) lp_spec = -2;  // not this slice's: prepare() loads it again
-  const int sel_tiles = (e_end - e_begin + kPagesPerTile - 1) / kPagesPerTile;
-  const int num_tiles = sel_tiles + (blk_cta ? plan.blk_tiles : 0);
-
-  pol.idx_row = idx_row;
-  pol.page_row = sh.page_table ? sh.page_table + (size_t)s * sh.max_pages : nullptr;
-  pol.q_head = a.q + ((size_t)s * sh.B * sh.Hq + (size_t)h * sh.G) * D;
-  pol.status = a.status;
-  pol.tab = nullptr;
-  pol.masks = nullptr;
-  pol.tab_off = M::table_offset();
-  pol.mask_off = M::mask_offset(plan.ppc);
-  pol.lp_spec = lp_spec;
-  pol.n_phys = sh.n_phys;
-  pol.phys0 = (long long)s * sh.max_pages;
-  pol.Hkv = sh.Hkv;
-  pol.h = h;
-  pol.G = sh.G;
-  pol.Hq = sh.Hq;
-  pol.B = sh.B;
-  pol.BG = sh.BG;
-  pol.s = s;
-  pol.n = n;
-  pol.np = (n + PAGE - 1) / PAGE;
-  pol.e_begin = e_begin;
-  pol.e_end = e_end;
-  pol.sel_tiles = sel_tiles;
-  pol.row_base = row_base;
-  pol.sl2 = sh.sl2;
-  eng.init(a.status, pol, num_tiles);
+  if (!early) key_side();
+  eng.init(a.status, pol, num_tiles, early && !blk_cta);
   // rows this CTA owns in the merge
   const int rpc = (kRowsPerCta + C - 1) / C;
   const int r0 = c * rpc;
@@ -583,19 +598,31 @@ inline int choose_page_ctas(const int *active, int nclusters, int kmax, int page
   return best;
 }
 
-template <int D, int PAGE>
-cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan_in, const SparseArgs &a,
-                         cudaStream_t stream) {
-  using M = SparseLayout<D>;
-  constexpr auto kern = sparse_attn<D, PAGE>;
-  constexpr size_t kMaxSmem = 227 * 1024;
-  cudaError_t err = set_smem_once<kern>(kMaxSmem);
+constexpr size_t kMaxSmem = 227 * 1024;
+
+// Kernel attributes set once per device: the dynamic shared memory and clusters
+// beyond the portable 8 CTAs.
+template <auto K>
+cudaError_t prepare_kernel_once() {
+  cudaError_t err = set_smem_once<K>(kMaxSmem);
   if (err != cudaSuccess) return err;
-  SparsePlan plan = plan_in;
-  const int *active = active_clusters<kern>(M::smem(std::max(sh.kmax, 64)));
-  const int cp = choose_page_ctas(active, sh.Hkv * sh.S * plan.rowtiles, sh.kmax, PAGE, plan.blk_tiles);
-  plan.cluster = cp + 1;
-  plan.ppc = (sh.kmax + cp - 1) / cp;
+  static unsigned long long done = 0;  // bit per device ordinal < 64
+  int dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (__atomic_load_n(&done, __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+  err = cudaFuncSetAttribute(K, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (err == cudaSuccess && bit) __atomic_fetch_or(&done, bit, __ATOMIC_ACQ_REL);
+  return err;
+}
+
+template <int D, int PAGE, int STG>
+cudaError_t launch_staged(const Shape &sh, const SparsePlan &plan, const SparseArgs &a,
+                          cudaStream_t stream) {
+  using M = SparseLayout<D, STG>;
+  constexpr auto kern = sparse_attn<D, PAGE, STG>;
+  cudaError_t err = prepare_kernel_once<kern>();
+  if (err != cudaSuccess) return err;
   const size_t smem = M::smem(plan.ppc);
   if (smem > kMaxSmem) return cudaErrorInvalidValue;
   CUtensorMap kmap, vmap, kmap4, vmap4, bkmap, bvmap;
@@ -633,6 +660,25 @@ cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan_in, const Spars
   return cudaGetLastError();
 }
 
+// Cluster shape from the device's cluster capacity, then the stage count: with
+// early gathering a page CTA holds all its tiles at once when they fit in four
+// stages; otherwise two stages stream them.
+template <int D, int PAGE>
+cudaError_t launch_typed(const Shape &sh, const SparsePlan &plan_in, const SparseArgs &a,
+                         cudaStream_t stream) {
+  constexpr auto probe = sparse_attn<D, PAGE, 2>;
+  cudaError_t err = prepare_kernel_once<probe>();
+  if (err != cudaSuccess) return err;
+  SparsePlan plan = plan_in;
+  const int *active = active_clusters<probe>(SparseLayout<D, 2>::smem(std::max(sh.kmax, 64)));
+  const int cp = choose_page_ctas(active, sh.Hkv * sh.S * plan.rowtiles, sh.kmax, PAGE, plan.blk_tiles);
+  plan.cluster = cp + 1;
+  plan.ppc = (sh.kmax + cp - 1) / cp;
+  const int tiles = (plan.ppc * PAGE + tc::kBN - 1) / tc::kBN;
+  if (sh.early_gather && tiles > 2) return launch_staged<D, PAGE, 4>(sh, plan, a, stream);
+  return launch_staged<D, PAGE, 2>(sh, plan, a, stream);
+}
+
 }  // namespace
 
 DSA_TRACE_EXPORT(dsa_trace_sparse)
@@ -651,6 +697,8 @@ SparsePlan plan_sparse(const Shape &sh, int /*num_sms*/) {
 
 cudaError_t launch_sparse(const Shape &sh, const SparsePlan &plan, const SparseArgs &a,
                           cudaStream_t stream) {
+  cudaError_t err = cudaSuccess;
+  if (launch_sparse_resident(sh, a, stream, &err)) return err;
   if (sh.d == 128) {
     if (sh.P == 16) return launch_typed<128, 16>(sh, plan, a, stream);
     if (sh.P == 32) return launch_typed<128, 32>(sh, plan, a, stream);

@@ -150,15 +150,32 @@ struct Engine {
     }
   }
 
+  // The key side of the set-up, for a policy whose tile addresses need no
+  // barrier (kIssueBeforeSync): the policy's per-CTA tables and the producer's
+  // loads of the first min(STAGES, num_tiles) tiles.  All threads call it; a
+  // kernel that may read the key side before its dependency wait calls it there,
+  // then init() with staged = true.
+  template <class Policy>
+  __device__ __forceinline__ void stage(Policy &pol, int num_tiles) {
+    static_assert(Policy::kIssueBeforeSync, "staging needs tables that warp 0 builds itself");
+    pol.prepare(smem);
+    if (threadIdx.x == 0) DSA_TRACE_EVENT(35);
+    if (warp == 0 && num_tiles > 0) issue_first(pol, num_tiles);
+  }
+
   // The data part of the set-up, after setup(): the policy's per-CTA tables, the
   // query rows copied by the softmax threads into the Q tile, and (for a policy
   // that allows it) the producer's loads of the first STAGES tiles, all before
-  // the CTA-wide barrier.
+  // the CTA-wide barrier.  With staged = true, stage() has already built the
+  // tables and issued those loads.
   template <class Policy>
-  __device__ __forceinline__ void init(uint32_t *status, Policy &pol, int num_tiles) {
+  __device__ __forceinline__ void init(uint32_t *status, Policy &pol, int num_tiles,
+                                       bool staged = false) {
     using namespace sm100;
-    pol.prepare(smem);  // per-CTA tables of the policy (all threads)
-    if (threadIdx.x == 0) DSA_TRACE_EVENT(35);
+    if (!staged) {
+      pol.prepare(smem);  // per-CTA tables of the policy (all threads)
+      if (threadIdx.x == 0) DSA_TRACE_EVENT(35);
+    }
     if (warp >= 2) {    // half of this row's query into the swizzled Q tile (zeros past the end)
       const int r = row_in_tile();
       constexpr int kChunks = D / 16;  // 16-byte chunks per half row
@@ -175,8 +192,8 @@ struct Engine {
       }
       fence_proxy_async_smem();
     }
-    // thread 0 is the producer: the first tiles' loads go out right away
-    if (Policy::kIssueBeforeSync && warp == 0 && num_tiles > 0) issue_first(pol, num_tiles);
+    // warp 0 is the producer: the first tiles' loads go out right away
+    if (!staged && Policy::kIssueBeforeSync && warp == 0 && num_tiles > 0) issue_first(pol, num_tiles);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -34,7 +34,7 @@ cudaError_t make_kv_tensor_map(CUtensorMap *out, const void *base, long long row
                                int box_rows) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
-  if (rows <= 0 || rows >= (1LL << 32)) return cudaErrorInvalidValue;
+  if (rows <= 0 || rows >= (1LL << 31)) return cudaErrorInvalidValue;  // int32 box coordinates
   cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)D * 2};
   cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
@@ -63,15 +63,36 @@ cudaError_t make_kv_pages_tensor_map(CUtensorMap *out, const void *base, long lo
 }
 
 // The block's own keys or values [S*B, Hkv, D] bf16 as a 3-D tensor (D, Hkv,
-// S*B); one box is 64 elements x 1 head x 64 tokens, so one load brings up to 64
-// consecutive tokens of one KV head (rows past S*B read as zeros).
+// S*B); one box is 64 elements x 1 head x `box_tokens` tokens (64 by default), so
+// one load brings up to that many consecutive tokens of one KV head (rows past
+// S*B read as zeros).
 cudaError_t make_blk_tensor_map(CUtensorMap *out, const void *base, long long tokens, int Hkv,
-                                int D) {
+                                int D, int box_tokens) {
   auto fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
+  if (box_tokens < 1 || box_tokens > 256) return cudaErrorInvalidValue;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)tokens};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
-  cuuint32_t box[3] = {64u, 1u, 64u};
+  cuuint32_t box[3] = {64u, 1u, (cuuint32_t)box_tokens};
+  cuuint32_t elem_strides[3] = {1u, 1u, 1u};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The block's queries [S*B, Hq, D] bf16 as a 3-D tensor (D, Hq, S*B); one box is
+// 64 elements x G heads x `tokens` tokens: the rows (b, g) of one KV head's group
+// for `tokens` consecutive tokens, landing as tokens*G rows of 128 bytes in the
+// order b*G + g (rows past S*B read as zeros).
+cudaError_t make_q_tensor_map(CUtensorMap *out, const void *base, long long tokens, int Hq, int D,
+                              int G, int box_tokens) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (G < 1 || G > 256 || box_tokens < 1 || box_tokens > 256) return cudaErrorInvalidValue;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+  cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)box_tokens};
   cuuint32_t elem_strides[3] = {1u, 1u, 1u};
   CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                   box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -33,7 +33,7 @@ EXPORTED = ("dsa_select", "dsa_sparse_attn", "dsa_select_workspace_size",
             "dsa_sparse_workspace_size", "dsa_workspace_init", "dsa_get_status",
             "dsa_strerror", "dsa_kernels_per_call", "dsa_select_launches", "dsa_version",
             "dsa_select_static_scratch",
-            "dsa_merge_attn")
+            "dsa_merge_attn", "dsa_sparse_kernel")
 
 
 class DsaError(RuntimeError):
@@ -49,7 +49,8 @@ class dsa_dims(ctypes.Structure):
                 ("n_phys", ctypes.c_int64), ("page_table", ctypes.c_void_p),
                 ("sm_limit", ctypes.c_int32), ("lse_out", ctypes.c_void_p),
                 ("head_budget", ctypes.c_int32), ("active", ctypes.c_void_p),
-                ("prefix_o_cache", ctypes.c_void_p), ("prefix_lse_cache", ctypes.c_void_p)]
+                ("prefix_o_cache", ctypes.c_void_p), ("prefix_lse_cache", ctypes.c_void_p),
+                ("early_gather", ctypes.c_int32)]
 
 
 _lib = None
@@ -91,6 +92,8 @@ def load(path: str = LIB_PATH):
     lib.dsa_kernels_per_call.argtypes = [ci]
     lib.dsa_select_launches.restype = ci
     lib.dsa_select_launches.argtypes = [dims_p]
+    lib.dsa_sparse_kernel.restype = ci
+    lib.dsa_sparse_kernel.argtypes = [dims_p]
     _lib = lib
     return lib
 
@@ -109,6 +112,15 @@ def select_launches(dims: dsa_dims) -> int:
     return rc
 
 
+def sparse_kernel(dims: dsa_dims) -> int:
+    """1 = streaming sparse kernel, 1 + C = the all-keys-resident kernel in clusters of
+    C CTAs, for these dims on the current device."""
+    rc = int(load().dsa_sparse_kernel(ctypes.byref(dims)))
+    if rc < 0:
+        raise DsaError(rc, "dsa_sparse_kernel")
+    return rc
+
+
 def strerror(code: int) -> str:
     return load().dsa_strerror(int(code)).decode()
 
@@ -123,10 +135,10 @@ def _stream(stream):
 
 
 def make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table=None,
-              sm_limit=0, head_budget=0) -> dsa_dims:
+              sm_limit=0, head_budget=0, early_gather=0) -> dsa_dims:
     return dsa_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys,
                     None if page_table is None else page_table.data_ptr(), int(sm_limit), None,
-                    int(head_budget), None, None, None)
+                    int(head_budget), None, None, None, int(early_gather))
 
 
 def _with_lse(dims: dsa_dims, lse_out) -> dsa_dims:
@@ -140,13 +152,13 @@ def _with_lse(dims: dsa_dims, lse_out) -> dsa_dims:
 
 
 def dims_for(q_blk, k_cache, max_pages, kmax, page_table=None, sm_limit=0,
-             head_budget=0) -> dsa_dims:
+             head_budget=0, early_gather=0) -> dsa_dims:
     S, B, Hq, d = q_blk.shape
     n_phys, Hkv, page, d2 = k_cache.shape
     if d2 != d:
         raise ValueError("q_blk and k_cache disagree on the head dimension")
     return make_dims(S, B, Hq, Hkv, d, page, max_pages, kmax, n_phys, page_table, sm_limit,
-                     head_budget)
+                     head_budget, early_gather)
 
 
 def _check(t, name, dtype, ndim=None):
@@ -281,9 +293,10 @@ def dsa_merge_attn(o_a, lse_a, o_b, lse_b, o_out, lse_out=None, stream=None):
 class DeviceWorkload:
     """A workload's tensors on the GPU plus the dims, outputs and workspaces of both passes."""
 
-    def __init__(self, w, device="cuda", sm_limit=0, head_budget=0):
+    def __init__(self, w, device="cuda", sm_limit=0, head_budget=0, early_gather=0):
         """head_budget=1: one budget of Hkv*kp pages per sequence shared by its KV heads;
-        idx rows then hold up to min(max_pages, Hkv*kp) pages."""
+        idx rows then hold up to min(max_pages, Hkv*kp) pages.  early_gather=1: sparse steps
+        gather their pages before waiting for the kernel ahead of them (include/dsa.h)."""
         self.w = w
         dev = torch.device(device)
         self.q1 = w.q1.to(dev)
@@ -297,7 +310,7 @@ class DeviceWorkload:
         kmax = min(w.max_pages, w.Hkv * w.kmax) if head_budget else w.kmax
         self.kmax = kmax
         self.dims = dims_for(self.q1, self.k_cache, w.max_pages, kmax, self.page_table, sm_limit,
-                             head_budget)
+                             head_budget, early_gather)
         S, Hkv = w.S, w.Hkv
         self.idx = torch.full((S, Hkv, kmax), -1, dtype=torch.int32, device=dev)
         self.cnt = torch.zeros((S, Hkv), dtype=torch.int32, device=dev)

@@ -120,6 +120,22 @@ typedef struct dsa_dims {
   float *prefix_lse_cache; /* with active: device fp32 [S, B, Hq]: its log-sum-exp, natural log
                          (-inf: no prefix key).  A stable row reads whatever its cache holds:
                          fill the caches with a call whose tokens are all active first. */
+  int32_t early_gather; /* sparse pass: 0 = read nothing the caller passes before the kernel
+                         launched just before this one on `stream` has completed; 1 = gather
+                         the selected pages early.  Every dsa_sparse_attn kernel is a
+                         programmatic dependent launch, so its CTAs can start while that
+                         preceding kernel still runs.  With early_gather = 1 they read n_ctx,
+                         idx_cnt, idx, the page table, k_cache and v_cache in that time and
+                         load the selected pages into shared memory; only q_blk, blk_k,
+                         blk_v (and o_out, lse_out, the workspace) wait for the preceding
+                         kernel.  CONTRACT: the kernel launched immediately before the call on
+                         the same stream writes none of n_ctx, idx_cnt, idx, page_table,
+                         k_cache, v_cache.  That holds when the page set is reused over a
+                         block's denoising steps (MAGE page, Approach) and the prefix cache
+                         is not appended to by that kernel: the indices come from a selection
+                         pass that ended before (on another stream, joined by an event, which
+                         orders it fully).  Work that is not a kernel (a copy, an event wait)
+                         is always fully ordered.  Ignored (treated as 0) with `active`. */
 } dsa_dims;
 
 /* cudaStream_t without including the CUDA headers. */
@@ -162,6 +178,9 @@ int dsa_select(const void *q_blk, const void *k_cache, const void *v_cache,
  * with no mask inside the block (bidirectional, self included).  idx entries
  * must be distinct logical pages below ceil(n_ctx[s]/page); an entry outside
  * that range is skipped and reported as DSA_ERR_BAD_INDEX through the status word.
+ * Launches: one kernel, a programmatic dependent of the kernel ahead of it on
+ * `stream` (see dims->early_gather).  Thread-block clusters split each (sequence,
+ * KV head)'s keys; dsa_sparse_kernel() tells which of the two kernels runs.
  */
 int dsa_sparse_attn(const void *q_blk, const void *k_cache, const void *v_cache,
                     const int32_t *idx, const void *blk_k, const void *blk_v,
@@ -261,6 +280,15 @@ const char *dsa_strerror(int code);
  * (DSA_ERR_INVALID_ARG otherwise).  Useful when capturing calls into a CUDA
  * graph or counting launches. */
 int dsa_kernels_per_call(int pass);
+
+/* Which kernel dsa_sparse_attn runs for these dims on the current device:
+ *   1      the streaming kernel (a ring of 64-key tiles per CTA; prefix-part
+ *          reuse, or more selected pages than 16 CTAs of a cluster can hold);
+ *   1 + C  the kernel whose CTAs hold all their keys in shared memory at once
+ *          (at most 256 each), in thread-block clusters of C CTAs per
+ *          (sequence, KV head, row tile);
+ * or a negative DSA_ERR_* code for bad dims.  Both compute the same result. */
+int dsa_sparse_kernel(const dsa_dims *dims);
 
 /* Kernel launches of one dsa_select (or dsa_select_static_scratch) call with
  * these dims on the current device, or a negative DSA_ERR_* code for bad dims. */

@@ -36,6 +36,9 @@ CASES = {
     "budget_covers_prefix": ("8k", dict(n=1500, topk=2048)),
     "p32": ("8k", dict(n=4000, P=32, topk=512)),
     "p64_d64": ("tiny", dict(n=3000, P=64, topk=256, B=8, Hq=8, Hkv=2)),
+    # more selected pages than the all-keys-resident kernel's CTAs can hold: the
+    # streaming kernel serves it
+    "wide_budget": ("8k", dict(n=8000, topk=8192)),
 }
 
 
@@ -43,8 +46,8 @@ def kp_list(w):
     return [int(w.topk[s]) // w.P for s in range(w.S)]
 
 
-def run_case(dsa_mod, w, steps=(2,), sm_limit=0):
-    dw = dsa_mod.DeviceWorkload(w, sm_limit=sm_limit)
+def run_case(dsa_mod, w, steps=(2,), sm_limit=0, early_gather=0):
+    dw = dsa_mod.DeviceWorkload(w, sm_limit=sm_limit, early_gather=early_gather)
     dw.select()
     torch.cuda.synchronize()
     assert dw.ws_sel.status() == dsa_mod.DSA_OK
@@ -82,7 +85,74 @@ def test_parity_with_sm_limit(dsa_mod, name, sm_limit):
 @pytest.mark.parametrize("name", ["128k", "batched"])
 def test_parity_full_size(dsa_mod, name):
     """Full-size workloads in the launch configuration the bench times."""
-    run_case(dsa_mod, W.make(name, 0), steps=(2,))
+    run_case(dsa_mod, W.make(name, 0), steps=(2,), early_gather=1)
+
+
+EARLY_CASES = ["tiny", "tiny_tail_d64", "8k", "32k_g7_p64", "ragged_paged", "kp1",
+               "budget_covers_prefix", "p64_d64", "wide_budget"]
+
+
+@pytest.mark.parametrize("case,resident", [("tiny", True), ("8k", True), ("32k_g7_p64", True),
+                                           ("ragged_paged", True), ("p64_d64", True),
+                                           ("wide_budget", False)])
+def test_sparse_kernel_choice(dsa_mod, case, resident):
+    """Which sparse kernel serves a shape (dsa_sparse_kernel): the all-keys-resident
+    kernel for the workloads' budgets, the streaming one past 16 CTAs x 256 keys or
+    with prefix-part reuse; the parity tests above then cover both."""
+    name, kw = CASES[case]
+    w = W.make(name, 0, **kw)
+    dw = dsa_mod.DeviceWorkload(w)
+    got = dsa_mod.sparse_kernel(dw.dims)
+    assert (got > 1) == resident, got
+    if resident:
+        on = torch.ones((w.S, w.B), dtype=torch.uint8, device="cuda")
+        d = dsa_mod.dsa_dims.from_buffer_copy(dw.dims)
+        d.active = on.data_ptr()
+        assert dsa_mod.sparse_kernel(d) == 1
+
+
+@pytest.mark.parametrize("name", ["128k", "batched"])
+def test_sparse_kernel_choice_full_size(dsa_mod, name):
+    w = W.make(name, 0)
+    dw = dsa_mod.DeviceWorkload(w)
+    assert dsa_mod.sparse_kernel(dw.dims) > 1
+
+
+@pytest.mark.parametrize("case", EARLY_CASES, ids=EARLY_CASES)
+def test_parity_early_gather(dsa_mod, case):
+    """dims.early_gather = 1: the pages are gathered before the dependency wait."""
+    name, kw = CASES[case]
+    run_case(dsa_mod, W.make(name, 0, **kw), steps=(2, 3), early_gather=1)
+
+
+@pytest.mark.parametrize("case", ["8k", "ragged_paged", "128k", "batched"])
+def test_early_gather_back_to_back(dsa_mod, case):
+    """Sparse steps of two layers queued back to back on one stream (each kernel a
+    programmatic dependent of the one before, so each gathers its pages while the
+    previous step still runs), every output against the oracle."""
+    name, kw = CASES.get(case, (case, {}))
+    ws = [W.make(name, seed, **kw) for seed in (0, 1)]
+    dws = [dsa_mod.DeviceWorkload(w, early_gather=1) for w in ws]
+    for dw in dws:
+        dw.select()
+    torch.cuda.synchronize()
+    steps = (2, 3, 4)
+    inputs = [[tuple(x.cuda() for x in w.step_inputs(t)) for t in steps] for w in ws]
+    outs = [[torch.empty_like(dw.q1) for _ in steps] for dw in dws]
+    for i in range(len(steps)):
+        for li, dw in enumerate(dws):
+            dw.sparse(*inputs[li][i], out=outs[li][i])
+    torch.cuda.synchronize()
+    for li, (w, dw) in enumerate(zip(ws, dws)):
+        assert dw.ws_sp.status() == dsa_mod.DSA_OK
+        pt = None if w.page_table is None else w.page_table.numpy()
+        gidx, gcnt = dw.idx.cpu().numpy(), dw.cnt.cpu().numpy()
+        for i, t in enumerate(steps):
+            q, bk, bv = w.step_inputs(t)
+            ref_o, _ = oracle.sparse(W.bits(q), W.bits(w.k_cache), W.bits(w.v_cache),
+                                     w.n_ctx.numpy(), gidx, gcnt, W.bits(bk), W.bits(bv),
+                                     page_table=pt, max_pages=w.max_pages)
+            parity.check_output(outs[li][i], ref_o, f"{w.name} layer {li} step {t}")
 
 
 def test_planted_needles_selected(dsa_mod):
@@ -152,6 +222,70 @@ def test_selection_on_second_stream(dsa_mod):
     torch.cuda.synchronize()
     assert torch.equal(dw.idx, idx_ref)
     assert torch.equal(o, o_ref)
+
+
+@pytest.mark.parametrize("case", ["8k", "ragged_paged"])
+def test_selection_stream_overlap_against_oracle(dsa_mod, case):
+    """The bench's step shape, checked against the oracle: for two layers, the
+    selection of block n+1 runs on a side stream while block n's sparse steps run on
+    the main stream (early gathering on, ping-pong index buffers); then block n+1's
+    first sparse step waits for the selection's event.  Every selection and every
+    sparse output is compared with the oracle."""
+    name, kw = CASES[case]
+    ws = [W.make(name, seed, **kw) for seed in (0, 1)]
+    dws = [dsa_mod.DeviceWorkload(w, early_gather=1) for w in ws]
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    idx = [[torch.full_like(dw.idx, -1) for _ in range(2)] for dw in dws]
+    cnt = [[torch.zeros_like(dw.cnt) for _ in range(2)] for dw in dws]
+    o_sel = [torch.empty_like(dw.q1) for dw in dws]
+    # block n's indices, then block n+1's queries (another step's draw stands in)
+    q_next = [w.step_inputs(9)[0] for w in ws]
+    for li, dw in enumerate(dws):
+        dw.select()
+        idx[li][0].copy_(dw.idx)
+        cnt[li][0].copy_(dw.cnt)
+    torch.cuda.synchronize()
+    steps = (2, 3, 4)
+    inputs = [[tuple(x.cuda() for x in w.step_inputs(t)) for t in steps] for w in ws]
+    qn = [q.cuda() for q in q_next]
+    outs = [[torch.empty_like(dw.q1) for _ in range(len(steps) + 1)] for dw in dws]
+    side.wait_stream(main)
+    with torch.cuda.stream(side):
+        for li, dw in enumerate(dws):
+            dsa_mod.dsa_select(qn[li], dw.k_cache, dw.v_cache, dw.n_ctx, dw.w.P, dw.topk,
+                               idx[li][1], o_sel[li], side, dims=dw.dims, cnt_out=cnt[li][1],
+                               workspace=dw.ws_sel)
+    ev = torch.cuda.Event()
+    ev.record(side)
+    for i in range(len(steps)):
+        for li, dw in enumerate(dws):
+            dw.sparse(*inputs[li][i], idx=idx[li][0], cnt=cnt[li][0], out=outs[li][i])
+    main.wait_event(ev)
+    for li, dw in enumerate(dws):   # block n+1, its first later step
+        dw.sparse(*inputs[li][0], idx=idx[li][1], cnt=cnt[li][1], out=outs[li][-1])
+    torch.cuda.synchronize()
+    for li, (w, dw) in enumerate(zip(ws, dws)):
+        assert dw.ws_sel.status() == dsa_mod.DSA_OK and dw.ws_sp.status() == dsa_mod.DSA_OK
+        pt = None if w.page_table is None else w.page_table.numpy()
+        ref_n = oracle.select(W.bits(w.q1), W.bits(w.k_cache), W.bits(w.v_cache), w.n_ctx.numpy(),
+                              w.topk.numpy(), page_table=pt, max_pages=w.max_pages)
+        ref_n1 = oracle.select(W.bits(q_next[li]), W.bits(w.k_cache), W.bits(w.v_cache),
+                               w.n_ctx.numpy(), w.topk.numpy(), page_table=pt,
+                               max_pages=w.max_pages)
+        npg = [w.n_pages(s) for s in range(w.S)]
+        gi0, gc0 = idx[li][0].cpu().numpy(), cnt[li][0].cpu().numpy()
+        gi1, gc1 = idx[li][1].cpu().numpy(), cnt[li][1].cpu().numpy()
+        parity.check_selection(gi0, gc0, ref_n, npg, kp_list(w))
+        parity.check_selection(gi1, gc1, ref_n1, npg, kp_list(w))
+        parity.check_output(o_sel[li], ref_n1.o, f"{w.name} layer {li} side-stream selection")
+        for i, t in enumerate(steps + (steps[0],)):
+            gi, gc = (gi0, gc0) if i < len(steps) else (gi1, gc1)
+            q, bk, bv = w.step_inputs(t)
+            ref_o, _ = oracle.sparse(W.bits(q), W.bits(w.k_cache), W.bits(w.v_cache),
+                                     w.n_ctx.numpy(), gi, gc, W.bits(bk), W.bits(bv),
+                                     page_table=pt, max_pages=w.max_pages)
+            parity.check_output(outs[li][i], ref_o, f"{w.name} layer {li} output {i}")
 
 
 def test_deterministic(dsa_mod):
