@@ -111,7 +111,7 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms in the background."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -125,7 +125,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -203,18 +203,30 @@ def max_over_ranks(x: float, world: int) -> float:
 
 
 # ----------------------------------------------------------------- CPU baseline
-def oracle_block(w, steps):
-    """The fp64 oracle on one block of one layer: selection + `steps` sparse steps."""
+def oracle_block(w, steps, seqs=None):
+    """The fp64 oracle on one block of one layer: selection + `steps` sparse steps, for
+    the first `seqs` sequences of the batch (all by default).  Returns the seconds."""
     import oracle
-    pt = None if w.page_table is None else w.page_table.numpy()
+    S = w.S if seqs is None else min(seqs, w.S)
+    pt = None if w.page_table is None else w.page_table.numpy()[:S]
+    n_ctx, topk = w.n_ctx.numpy()[:S], w.topk.numpy()[:S]
+    inputs = [tuple(x[:S] for x in w.step_inputs(t)) for t in range(2, 2 + steps)]
     t0 = time.perf_counter()
-    r = oracle.select(W.bits(w.q1), W.bits(w.k_cache), W.bits(w.v_cache), w.n_ctx.numpy(),
-                      w.topk.numpy(), page_table=pt, max_pages=w.max_pages)
-    for t in range(2, 2 + steps):
-        q, bk, bv = w.step_inputs(t)
-        oracle.sparse(W.bits(q), W.bits(w.k_cache), W.bits(w.v_cache), w.n_ctx.numpy(), r.idx,
-                      r.cnt, W.bits(bk), W.bits(bv), page_table=pt, max_pages=w.max_pages)
+    r = oracle.select(W.bits(w.q1[:S]), W.bits(w.k_cache), W.bits(w.v_cache), n_ctx, topk,
+                      page_table=pt, max_pages=w.max_pages)
+    for q, bk, bv in inputs:
+        oracle.sparse(W.bits(q), W.bits(w.k_cache), W.bits(w.v_cache), n_ctx, r.idx, r.cnt,
+                      W.bits(bk), W.bits(bv), page_table=pt, max_pages=w.max_pages)
     return time.perf_counter() - t0
+
+
+def sample_bytes(w, steps, seqs=None):
+    """Algorithmic bytes of oracle_block's sample."""
+    S = w.S if seqs is None else min(seqs, w.S)
+    kv = sum(int(w.n_ctx[s]) for s in range(S)) * w.Hkv * w.d * 2 * 2
+    sel = sum(min(int(w.topk[s]), w.n_pages(s) * w.P) for s in range(S)) * w.Hkv * w.d * 2 * 2
+    qo = 2 * S * w.B * w.Hq * w.d * 2
+    return kv + qo + steps * (sel + qo)
 
 
 def block_time_shape(dsa, names=("8k", "32k", "128k"), reps=20):
@@ -257,14 +269,18 @@ def block_time_shape(dsa, names=("8k", "32k", "128k"), reps=20):
 
 
 def cpu_baseline(w):
+    """The oracle as it stands on the host cores: one block of one layer (the selection
+    pass plus T-1 sparse steps); of a batch, its first sequence only (a bounded sample)."""
     import oracle
     steps = w.T - 1
-    secs = oracle_block(w, steps)
-    nbytes = select_bytes(w) + steps * sparse_bytes(w)
+    seqs = 1 if w.S > 1 else None
+    secs = oracle_block(w, steps, seqs)
+    nbytes = sample_bytes(w, steps, seqs)
+    what = "its first sequence" if seqs else "the whole workload"
     return {"value": round(nbytes / secs / 1e9, 6), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"one block of one layer of the {w.name} workload: the selection pass "
-                      f"plus {steps} sparse steps ({nbytes} algorithmic bytes) in {secs:.2f} s"}
+            "kind": "oracle", "seconds": round(secs, 3),
+            "sample": f"one block of one layer of the {w.name} workload ({what}): the selection "
+                      f"pass plus {steps} sparse steps ({nbytes} algorithmic bytes) in {secs:.2f} s"}
 
 
 def run_reference(args, world, rank):
@@ -299,12 +315,14 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ GPU bench
 class Bench:
-    def __init__(self, w, layers: int, dsa):
+    def __init__(self, w, layers: int, dsa, select_sms: int = 0):
         self.w, self.L, self.dsa = w, layers, dsa
         dev = torch.device("cuda")
         T, S = w.T, w.S
         self.main = torch.cuda.current_stream()   # a non-default stream set by run_ours
-        self.side = torch.cuda.Stream()
+        self.side = torch.cuda.Stream()           # the selection of the next block
+        self.h2d = torch.cuda.Stream()            # end-to-end runs: inputs in, ahead of use
+        self.d2h = torch.cuda.Stream()            # end-to-end runs: outputs out, behind
         # L independent layer copies of the KV cache
         self.k = torch.empty((layers, *w.k_cache.shape), dtype=torch.bfloat16, device=dev)
         self.v = torch.empty_like(self.k)
@@ -326,14 +344,17 @@ class Bench:
         # the sparse steps reuse indices the selection wrote one block earlier (on the side
         # stream, joined by an event): each gathers its pages before the kernel ahead of it ends
         self.dims = dsa.dims_for(self.q[0, 0], self.k[0], w.max_pages, w.kmax, self.page_table,
-                                 early_gather=1)
+                                 sm_limit=select_sms, early_gather=1)
         self.idx = torch.full((2, layers, S, w.Hkv, w.kmax), -1, dtype=torch.int32, device=dev)
         self.cnt = torch.zeros((2, layers, S, w.Hkv), dtype=torch.int32, device=dev)
         self.o_sel = torch.empty((layers, *w.q1.shape), dtype=torch.bfloat16, device=dev)
-        self.o_sp = torch.empty((layers, *w.q1.shape), dtype=torch.bfloat16, device=dev)
+        # one output per (layer, later step): an output copied to the host end to end
+        # is never overwritten by a later kernel
+        self.o_sp = torch.empty((layers, T - 1, *w.q1.shape), dtype=torch.bfloat16, device=dev)
         self.ws_sel = dsa.Workspace(dsa.select_workspace_size(self.dims), dev)
         self.ws_sp = dsa.Workspace(dsa.sparse_workspace_size(self.dims), dev)
         self.host_o = torch.empty((T, *w.q1.shape), dtype=torch.bfloat16).pin_memory()
+        self.host_o_sel = torch.empty(w.q1.shape, dtype=torch.bfloat16).pin_memory()
         self.host_idx = torch.empty((w.S, w.Hkv, w.kmax), dtype=torch.int32).pin_memory()
 
     # one call each -------------------------------------------------------------
@@ -344,32 +365,64 @@ class Bench:
 
     def sparse(self, l, t, buf, stream):
         self.dsa.dsa_sparse_attn(self.q[l, t], self.k[l], self.v[l], self.idx[buf, l],
-                                 self.bk[l, t], self.bv[l, t], self.o_sp[l], stream,
+                                 self.bk[l, t], self.bv[l, t], self.o_sp[l, t - 1], stream,
                                  dims=self.dims, n_ctx=self.n_ctx, idx_cnt=self.cnt[buf, l],
                                  workspace=self.ws_sp)
 
     # the block step: select(next) on the side stream || sparse(current) on main
     def block_step(self, cur, e2e=False):
         nxt = 1 - cur
-        self.side.wait_stream(self.main)
-        with torch.cuda.stream(self.side):
-            for l in range(self.L):
-                if e2e:
-                    self.q[l, 0].copy_(self.host_q[0], non_blocking=True)
-                self.select(l, nxt, self.side)
-                if e2e:
-                    self.host_o[0].copy_(self.o_sel[l], non_blocking=True)
-                    self.host_idx.copy_(self.idx[nxt, l], non_blocking=True)
-        for t in range(1, self.w.T):
-            for l in range(self.L):
-                if e2e:
+        L, T = self.L, self.w.T
+        main, side = self.main, self.side
+        if not e2e:
+            side.wait_stream(main)
+            with torch.cuda.stream(side):
+                for l in range(L):
+                    self.select(l, nxt, side)
+            for t in range(1, T):
+                for l in range(L):
+                    self.sparse(l, t, cur, main)
+            main.wait_stream(side)
+            return
+        # End to end: every call's inputs are copied in from pinned host memory on a
+        # copy stream, ahead of their use (an event per call gates it), and every
+        # output is copied back on another stream once its kernel is done, so that
+        # the copies overlap the kernels.
+        side.wait_stream(main)
+        self.h2d.wait_stream(main)
+        self.d2h.wait_stream(main)
+        ready = {}
+        with torch.cuda.stream(self.h2d):
+            for t in range(T):
+                for l in range(L):
                     self.q[l, t].copy_(self.host_q[t], non_blocking=True)
-                    self.bk[l, t].copy_(self.host_bk[t], non_blocking=True)
-                    self.bv[l, t].copy_(self.host_bv[t], non_blocking=True)
-                self.sparse(l, t, cur, self.main)
-                if e2e:
-                    self.host_o[t].copy_(self.o_sp[l], non_blocking=True)
-        self.main.wait_stream(self.side)
+                    if t > 0:
+                        self.bk[l, t].copy_(self.host_bk[t], non_blocking=True)
+                        self.bv[l, t].copy_(self.host_bv[t], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(self.h2d)
+                    ready[(l, t)] = ev
+        for l in range(L):
+            side.wait_event(ready[(l, 0)])
+            self.select(l, nxt, side)
+            done = torch.cuda.Event()
+            done.record(side)
+            self.d2h.wait_event(done)
+            with torch.cuda.stream(self.d2h):
+                self.host_o_sel.copy_(self.o_sel[l], non_blocking=True)
+                self.host_idx.copy_(self.idx[nxt, l], non_blocking=True)
+        for t in range(1, T):
+            for l in range(L):
+                main.wait_event(ready[(l, t)])
+                self.sparse(l, t, cur, main)
+                done = torch.cuda.Event()
+                done.record(main)
+                self.d2h.wait_event(done)
+                with torch.cuda.stream(self.d2h):
+                    self.host_o[t].copy_(self.o_sp[l, t - 1], non_blocking=True)
+        main.wait_stream(side)
+        main.wait_stream(self.h2d)
+        main.wait_stream(self.d2h)
 
     def h2d_d2h_bytes(self):
         w, L = self.w, self.L
@@ -421,56 +474,122 @@ def run_ours(args, world, rank, local):
         _run_ours(args, world, rank, local, dsa)
 
 
-def _run_ours(args, world, rank, local, dsa):
-    w = W.make(args.workload, 0)
-    b = Bench(w, args.layers, dsa)
-    hbm_peak, tc_peak, peak_kind = load_peaks()
-    T, L = w.T, args.layers
-    step_bytes = L * (select_bytes(w) + (T - 1) * sparse_bytes(w))
-    launches_per_step = L * (dsa.select_launches(b.dims) + (T - 1) * dsa.kernels_per_call(1))
+LAYERS = {"128k": 64, "8k": 64, "32k": 64, "tiny": 64, "batched": 4}
 
-    # initial selection (block 0's indices), eager warm-up of every kernel
-    for l in range(L):
+
+def measure(w, layers, dsa, steps, warmup, world, select_sms=0, clocks=None, e2e=False):
+    """The block step of workload `w` over `layers` independent layer copies: the
+    overlapped step (selection of the next block on the side stream, the T-1 sparse
+    steps of the current block on the main stream) captured in CUDA graphs and
+    replayed, then the selection alone and the sparse steps alone (their own graph),
+    and end to end if asked.  Times in ms / us from CUDA events on the launching
+    stream; the step time is the max over ranks."""
+    b = Bench(w, layers, dsa, select_sms)
+    T, L = w.T, layers
+    for l in range(L):  # block 0's indices; every kernel warmed up eagerly
         b.select(l, 0, b.main)
+    torch.cuda.synchronize()
     b.sparse(0, 1, 0, b.main)
     torch.cuda.synchronize()
-
     graphs = b.capture()
-    for i in range(args.warmup):
+    for i in range(warmup):
         graphs[i % 2].replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        ms = timed(lambda i: graphs[(args.warmup + i) % 2].replay(), args.steps, b.main)
+    if clocks is not None:
+        with clocks:
+            ms = timed(lambda i: graphs[(warmup + i) % 2].replay(), steps, b.main)
+    else:
+        ms = timed(lambda i: graphs[(warmup + i) % 2].replay(), steps, b.main)
     barrier(world)
     ms = max_over_ranks(ms, world)
+    del graphs
     status_sel, status_sp = b.ws_sel.status(), b.ws_sp.status()
     if status_sel != dsa.DSA_OK or status_sp != dsa.DSA_OK:
-        raise SystemExit(f"device status: select {status_sel}, sparse {status_sp}")
-
-    # phase timings (reported beside the headline): selection alone, sparse alone
+        raise SystemExit(f"{w.name}: device status: select {status_sel}, sparse {status_sp}")
+    # the parts alone: the selection (eager launches over the layers) and the
+    # sparse steps (their own graph)
     reps = 3
     sel_ms = timed(lambda i: [b.select(l, 0, b.main) for l in range(L)], reps, b.main) / L
+    torch.cuda.synchronize()
+    sel_full_ms = sel_ms
+    if select_sms:  # the pass alone on the whole device, as a caller without a second stream runs it
+        dims_sm = b.dims
+        b.dims = dsa.dims_for(b.q[0, 0], b.k[0], w.max_pages, w.kmax, b.page_table, early_gather=1)
+        b.ws_sel = dsa.Workspace(dsa.select_workspace_size(b.dims), "cuda")
+        for l in range(L):
+            b.select(l, 0, b.main)
+        sel_full_ms = timed(lambda i: [b.select(l, 0, b.main) for l in range(L)], reps, b.main) / L
+        torch.cuda.synchronize()
+        b.dims = dims_sm
     g_sp = b.capture_sparse_only()
     g_sp.replay()
     sp_us = 1e3 * timed(lambda i: g_sp.replay(), reps, b.main) / ((T - 1) * L)
     del g_sp
+    out = {"b": b, "ms": ms, "sel_ms": sel_ms, "sel_full_ms": sel_full_ms, "sp_us": sp_us,
+           "launches_per_step": L * (dsa.select_launches(b.dims) + (T - 1) * dsa.kernels_per_call(1)),
+           "sparse_kernel": dsa.sparse_kernel(b.dims), "select_sms": select_sms}
+    if e2e:
+        e2e_graphs = b.capture(e2e=True)
+        for i in range(2):
+            e2e_graphs[i % 2].replay()
+        out["e2e_ms"] = max_over_ranks(timed(lambda i: e2e_graphs[i % 2].replay(), steps, b.main), world)
+        del e2e_graphs
+        out["h2d"], out["d2h"] = b.h2d_d2h_bytes()
+    return out
 
-    # e2e: the same step with host<->device copies of every call's inputs/outputs
-    e2e_graphs = b.capture(e2e=True)
-    for i in range(2):
-        e2e_graphs[i % 2].replay()
-    e2e_ms = max_over_ranks(timed(lambda i: e2e_graphs[i % 2].replay(), args.steps, b.main), world)
-    del e2e_graphs
-    h2d, d2h = b.h2d_d2h_bytes()
+
+def config_entry(w, m, layers, hbm_peak, world, cpu):
+    """One workload's numbers for the JSON line (the headline's sub-objects use the
+    same fields)."""
+    T = w.T
+    sel_b, sp_b = select_bytes(w), sparse_bytes(w)
+    sel_gbs = sel_b / (m["sel_full_ms"] * 1e-3) / 1e9
+    sp_gbs = sp_b / (m["sp_us"] * 1e-6) / 1e9
+    serial = layers * (m["sel_ms"] + (T - 1) * m["sp_us"] * 1e-3)
+    e = {"workload": WORKLOAD_TEXT.get(w.name, w.name), "layers_rotated": layers,
+         "step_ms": round(m["ms"], 4),
+         "step_gbs": round(world * layers * (sel_b + (T - 1) * sp_b) / (m["ms"] * 1e-3) / 1e9, 1),
+         "sparse_step_us": round(m["sp_us"], 3), "sparse_step_gbs": round(sp_gbs, 1),
+         "sparse_frac": round(sp_gbs / hbm_peak, 4), "sparse_bytes": sp_b,
+         "sparse_kernel": ("resident, clusters of %d" % (m["sparse_kernel"] - 1)
+                           if m["sparse_kernel"] > 1 else "streaming"),
+         "select_pass_ms": round(m["sel_full_ms"], 4), "select_pass_gbs": round(sel_gbs, 1),
+         "select_pass_ms_in_step": round(m["sel_ms"], 4),
+         "select_frac": round(sel_gbs / hbm_peak, 4), "select_bytes": sel_b,
+         "overlap": {"what": f"makespan of the block step (the selection of the next block on a "
+                             f"second stream beside the {T - 1} sparse steps of the current one, "
+                             f"{layers} layers) against the sum of the parts timed alone",
+                     "select_sms": m["select_sms"] or "all",
+                     "serial_ms": round(serial, 4), "makespan_ms": round(m["ms"], 4),
+                     "gain": round(serial / m["ms"] - 1.0, 4)}}
+    if cpu:
+        e["oracle"] = cpu_baseline(w)
+    return e
+
+
+def _run_ours(args, world, rank, local, dsa):
+    w = W.make(args.workload, 0)
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+    T, L = w.T, args.layers
+    clk = ClockSampler(local)
+    m = measure(w, L, dsa, args.steps, args.warmup, world, args.select_sms, clocks=clk, e2e=True)
+    b, ms, sel_ms, sp_us = m["b"], m["ms"], m["sel_full_ms"], m["sp_us"]
+    step_bytes = L * (select_bytes(w) + (T - 1) * sparse_bytes(w))
+    launches_per_step = m["launches_per_step"]
+    e2e_ms, h2d, d2h = m["e2e_ms"], m["h2d"], m["d2h"]
+    head = config_entry(w, m, L, hbm_peak, world, cpu=False)
+    host_q = b.host_q
+    del m, b
+    torch.cuda.empty_cache()
 
     # MAGE's central quantity (outside the timed region): recall of the page set in
     # use at each step against that step's own top-k, for the reused step-1 set
     # and for a refresh every 8 steps
     from block_sparse_attention_27_b200 import recall as R
     dw = dsa.DeviceWorkload(w)
-    qs = [b.host_q[t].cuda() for t in range(T)]
+    qs = [host_q[t].cuda() for t in range(T)]
     rec_reused = R.step_recall(dw, qs)
     rec_anchor8 = R.step_recall(dw, qs, anchor=8)
     # exact step-1 output: what it costs beyond the selection pass (which writes its
@@ -516,6 +635,18 @@ def _run_ours(args, world, rank, local, dsa):
                                                        cache=(c_o, c_l)), 50, cur)
     del dw, dwh, qs, c_o, c_l
     shape = block_time_shape(dsa)
+    torch.cuda.empty_cache()
+
+    # the other workloads, timed the same way (each its own graphs over its own
+    # layer copies; the batched workload holds ~1.3 GB of cache per layer, so fewer)
+    configs = {}
+    for name in [c for c in args.configs.split(",") if c and c != "none" and c != args.workload]:
+        wc = W.make(name, 0)
+        mc = measure(wc, LAYERS.get(name, 64), dsa, args.steps, args.warmup, world, args.select_sms)
+        configs[name] = config_entry(wc, mc, LAYERS.get(name, 64), hbm_peak, world,
+                                     cpu=(world == 1 and not args.no_cpu_baseline))
+        del mc, wc
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return
@@ -533,6 +664,7 @@ def _run_ours(args, world, rank, local, dsa):
                            f"of the next block ({L} x dsa_select, second stream) overlapped with "
                            f"{T - 1} x {L} dsa_sparse_attn of the current block",
                    "layers_rotated": L,
+                   "select_sms": args.select_sms or "all",
                    "l2": f"inputs larger than L2: {L} distinct K/V caches, queries and outputs "
                          f"({step_bytes / 1e9:.1f} GB of algorithmic traffic per step)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
@@ -540,19 +672,28 @@ def _run_ours(args, world, rank, local, dsa):
         "sparse_step_gbs": round(sp_gbs, 1),
         "select_pass_ms": round(sel_ms, 4),
         "select_pass_gbs": round(sel_gbs, 1),
-        "roofline": {"bound": "hbm", "kernel": "selection pass (dsa_select)",
-                     "achieved": round(sel_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(sel_gbs / hbm_peak, 4),
-                     "traffic": recorded_traffic("select", args.workload),
-                     "algorithmic_bytes_per_launch": sel_b, "peak_kind": peak_kind},
-        "roofline_sparse": {"bound": "hbm", "kernel": "sparse step (dsa_sparse_attn)",
-                            "achieved": round(sp_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
-                            "frac": round(sp_gbs / hbm_peak, 4),
-                            "traffic": recorded_traffic("sparse", args.workload),
-                            "algorithmic_bytes_per_launch": sp_b, "peak_kind": peak_kind},
+        "select_pass_ms_in_step": head["select_pass_ms_in_step"],
+        # the kernel that takes most of the step: the sparse step
+        "roofline": {"bound": "hbm", "kernel": "sparse step (dsa_sparse_attn)",
+                     "achieved": round(sp_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(sp_gbs / hbm_peak, 4),
+                     "traffic": recorded_traffic("sparse", args.workload),
+                     "algorithmic_bytes_per_launch": sp_b, "peak_kind": peak_kind,
+                     "share_of_step": round(L * (T - 1) * sp_us * 1e-3 / ms, 3)},
+        "roofline_select": {"bound": "hbm", "kernel": "selection pass (dsa_select)",
+                            "achieved": round(sel_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                            "frac": round(sel_gbs / hbm_peak, 4),
+                            "traffic": recorded_traffic("select", args.workload),
+                            "algorithmic_bytes_per_launch": sel_b, "peak_kind": peak_kind,
+                            "timed": "alone on the whole device (one cooperative launch)"},
+        "overlap": head["overlap"],
+        "sparse_kernel": head["sparse_kernel"],
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h)},
+                "d2h_bytes_per_step": int(d2h),
+                "how": "inputs of every call copied in from pinned host memory on a copy stream "
+                       "ahead of use, every output copied back on another stream, inside the "
+                       "timed graphs"},
         "gpu_launches": int(launches_per_step * args.steps),
         "clocks": clk.summary(),
         "tensor_tflops_select": round(select_flops(w) / (sel_ms * 1e-3) / 1e12, 1),
@@ -581,9 +722,12 @@ def _run_ours(args, world, rank, local, dsa):
                                      "of sparse over exact attention at every step; eager launches",
                              **shape},
     }
+    line["configs"] = configs
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line, ensure_ascii=False), flush=True)
+
+
 
 
 def main():
@@ -595,6 +739,14 @@ def main():
     ap.add_argument("--workload", default="128k", choices=list(WORKLOAD_TEXT))
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", default="8k,32k,batched,tiny",
+                    help="other workloads timed the same way and reported under 'configs' "
+                         "(comma list, or 'none')")
+    ap.add_argument("--select-sms", type=int, default=64,
+                    help="SMs the selection pass may hold in the block step (dsa_dims.sm_limit; "
+                         "0 = all, one cooperative launch that holds the device).  64 gives "
+                         "groups of 8 CTAs launched as clusters, so that the selection of the "
+                         "next block runs beside the sparse steps")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

@@ -3,7 +3,8 @@
 // KV head ("MAGE: All-[MASK] Block Already Knows Where to Look in Block
 // Diffusion LLM", Approach).
 //
-// select_fused, launched cooperatively (all its CTAs co-resident).  A group is
+// select_fused, launched so that the CTAs of a group are co-resident (as one
+// thread-block cluster when a group has at most 16 CTAs, else cooperatively).  A group is
 // one (sequence, KV head); its CTAs are the (split, 128-row tile) pairs.
 //   1. Split-KV attention on the tcgen05 engine (tc_attn.cuh).  Per split: the
 //      unnormalised O_j with row max m_j and sum l_j; per (tile, row): the mass
@@ -1471,18 +1472,44 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
   constexpr size_t smem = tc::Layout<D, kSelStages>::kAlloc;
   err = set_smem_once<kern>(smem);
   if (err != cudaSuccess) return err;
-  // Cooperative: the CTAs of a launch are co-resident, which the group barrier
-  // needs.  Programmatic dependent: the set-up overlaps the tail of the kernel
-  // ahead on the stream.
+  // The group barrier needs the CTAs of a group co-resident.  A group of at most
+  // 16 CTAs is one thread-block cluster (co-scheduled by the hardware; groups do
+  // not wait for one another, so kernels of other streams run beside them); a
+  // larger group needs a cooperative launch, which holds the device for itself.
+  // The cooperative launch is also a programmatic dependent of the kernel ahead
+  // on the stream (its set-up overlaps that kernel's tail); the clustered one is
+  // not: a dependent's CTAs would take SMs while they wait, the SMs that the
+  // kernels of another stream use when the pass is held to part of the device
+  // (dsa_dims.sm_limit) to run beside them.
+  const bool clustered = plan.group_ctas <= 16;
+  if (clustered) {
+    static unsigned long long big_done = 0;  // bit per device ordinal < 64
+    int dev = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (!bit || !(__atomic_load_n(&big_done, __ATOMIC_ACQUIRE) & bit)) {
+      if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) !=
+          cudaSuccess)
+        return err;
+      if (bit) __atomic_fetch_or(&big_done, bit, __ATOMIC_ACQ_REL);
+    }
+  }
   cudaLaunchAttribute attrs[2];
-  attrs[0].id = cudaLaunchAttributeCooperative;
-  attrs[0].val.cooperative = 1;
-  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  if (clustered) {
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = plan.group_ctas;
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = 1;
+  } else {
+    attrs[1].id = cudaLaunchAttributeCooperative;
+    attrs[1].val.cooperative = 1;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.stream = stream;
-  cfg.attrs = attrs;
-  cfg.numAttrs = 2;
+  cfg.attrs = clustered ? attrs + 1 : attrs;
+  cfg.numAttrs = clustered ? 1 : 2;
   cfg.blockDim = dim3(tc::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   const int groups = sh.S * sh.Hkv;
@@ -1493,7 +1520,7 @@ cudaError_t launch_typed(const Shape &sh, const SelectPlan &plan, const SelectAr
     if (err != cudaSuccess) return err;
   }
   if (sh.head_budget) {  // the selection over all KV heads of each sequence
-    cfg.attrs = attrs + 1;  // programmatic dependent only
+    cfg.attrs = attrs;  // programmatic dependent only
     cfg.numAttrs = 1;
     err = set_smem_once<select_global_topk>(kGlobalSmem);
     if (err != cudaSuccess) return err;

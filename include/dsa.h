@@ -92,6 +92,10 @@ typedef struct dsa_dims {
   int32_t sm_limit;   /* selection pass: the most SMs its attention kernel may hold at once,
                          so that it can run on its own stream beside the sparse steps
                          (which then keep the other SMs); 0 = every SM of the device.
+                         When a (sequence, KV head)'s CTAs number at most 16 (the split
+                         count follows from the SMs), they are launched as one thread-block
+                         cluster and the pass shares the device with other streams;
+                         otherwise the pass is one cooperative launch that holds the device.
                          Workspace sizes depend on it: query them with the same dims. */
   float *lse_out;     /* optional device fp32 [S, B, Hq], NULL = not written: the call that
                          receives these dims stores, per query row, the natural log of the sum
