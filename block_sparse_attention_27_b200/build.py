@@ -45,9 +45,14 @@ def _deps():
 
 
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    return up_to_date_at(LIB)
+
+
+def up_to_date_at(lib: str) -> bool:
+    """True when `lib` exists and is newer than every source it is built from."""
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
@@ -57,7 +62,7 @@ def build(force: bool = False, verbose: bool = False, defines=(), out: str | Non
     lib = out or LIB
     if not force and not defines and out is None and up_to_date():
         return LIB
-    objdir = BUILD if out is None else os.path.join(os.path.dirname(out), "_obj")
+    objdir = BUILD if out is None else os.path.join(BUILD, os.path.splitext(os.path.basename(out))[0])
     os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
     extra = (["-Xptxas", "-v"] if verbose else []) + [f"-D{d}" for d in defines]

@@ -983,7 +983,10 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   const bool started = sc.flag;
   if (started && threadIdx.x == 0) st.start();
   if (threadIdx.x == 0) {
-    if (!sm100::wait_count_geq(arrive, (uint32_t)G)) sm100::note_timeout(a.status, 0xffu);
+    // (the test build waits for one arrival more than the group has, so that this
+    // wait runs out and reports itself; all G partials are written even then)
+    if (!sm100::wait_count_geq(arrive, (uint32_t)G + sm100::kTestExtraArrivals))
+      sm100::note_timeout(a.status, 0xffu);
     DSA_TRACE_EVENT(41);
   }
   sm100::fence_proxy_async_global();  // the other CTAs' partials, before the bulk copies

@@ -22,7 +22,15 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+#ifdef DSA_TEST_TIMEOUT
+// Test build only: a short limit, so that the test that makes a wait run out
+// (see kTestExtraArrivals) finishes quickly.
+constexpr uint64_t kWaitLimitNs = 50000000ull;  // 50 ms
+constexpr uint32_t kTestExtraArrivals = 1;
+#else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+constexpr uint32_t kTestExtraArrivals = 0;
+#endif
 
 // Shared state for bounded waits of one CTA.
 struct WaitCtx {

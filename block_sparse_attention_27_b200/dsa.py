@@ -57,10 +57,18 @@ _lib = None
 
 
 def load(path: str = LIB_PATH):
-    """Load libdsa.so (raises if it has not been built)."""
+    """Load libdsa.so (raises if it has not been built); the binding's functions use
+    the first library loaded."""
     global _lib
     if _lib is not None:
         return _lib
+    _lib = open_library(path)
+    return _lib
+
+
+def open_library(path: str):
+    """A libdsa build at `path` with the C ABI's signatures declared, independent of
+    the one the binding's functions use (e.g. a test build of the same sources)."""
     if not os.path.exists(path):
         raise RuntimeError(f"libdsa.so not built ({path}); run "
                            "`python -m block_sparse_attention_27_b200.build`")
@@ -94,7 +102,6 @@ def load(path: str = LIB_PATH):
     lib.dsa_select_launches.argtypes = [dims_p]
     lib.dsa_sparse_kernel.restype = ci
     lib.dsa_sparse_kernel.argtypes = [dims_p]
-    _lib = lib
     return lib
 
 
@@ -226,6 +233,8 @@ def dsa_select_static_scratch(q_blk, k_cache, v_cache, n_ctx, page, topk, idx_ou
     _check(idx_out, "idx_out", torch.int32)
     _check(o_out, "o_out", torch.bfloat16)
     _check(cnt_out, "cnt_out", torch.int32)
+    if status.dtype == torch.uint32:  # the same 4-byte word either way
+        status = status.view(torch.int32)
     _check(status, "status", torch.int32)
     rc = load().dsa_select_static_scratch(_ptr(q_blk), _ptr(k_cache), _ptr(v_cache), _ptr(n_ctx),
                                           int(page), _ptr(topk), _ptr(idx_out), _ptr(o_out),

@@ -207,8 +207,11 @@ int dsa_workspace_init(void *workspace, size_t ws_bytes, dsa_stream_t stream);
  * DSA_ERR_DEVICE_TIMEOUT, bits 16..31 of the word (read it directly) identify the
  * first wait that gave up: bits 16..23 its barrier's shared-memory address / 8
  * (mod 256), or 255 for the selection pass's wait on the other CTAs of its
- * (sequence, KV head); bits 24..31 the waiting warp.  A workspace whose call
- * timed out must be zeroed again with dsa_workspace_init() before its next use. */
+ * (sequence, KV head); bits 24..31 the waiting warp.  The word is sticky: clear
+ * it with dsa_workspace_init() (for dsa_select_static_scratch, write 0 to the
+ * caller's status word).  Nothing else needs resetting after a wait ran out: the
+ * selection pass's group counters return to zero at the end of every call, since
+ * every CTA still reaches it. */
 int dsa_get_status(const void *workspace, dsa_stream_t stream);
 
 /*

@@ -52,6 +52,25 @@ def test_static_scratch_matches_workspace_path(names):
     assert int(status.item()) == 0
 
 
+@pytest.mark.parametrize("kw", [dict(head_budget=1), dict(sm_limit=4)],
+                         ids=["head_budget", "sm_limit"])
+def test_static_scratch_variants(kw):
+    """The head-adaptive budget (whose second kernel reads the page scores from the
+    array) and a pass held to 4 SMs (two selection launches reusing the group
+    counters of one call), each twice in a row, equal to dsa_select."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dw = dsa.DeviceWorkload(W.make("8k", 0), **kw)
+    assert dsa.select_workspace_size(dw.dims) <= dsa.DSA_SELECT_STATIC_SCRATCH_BYTES
+    q2 = dw.w.step_inputs(2)[0].cuda()
+    for q in (dw.q1, q2, dw.q1):
+        want = tuple(t.clone() for t in dw.select(q))
+        got = _static_select(dw, q, status)
+        torch.cuda.synchronize()
+        _compare(dw, got, want)
+    assert dw.ws_sel.status() == dsa.DSA_OK
+    assert dsa.status_word(status) == dsa.DSA_OK
+
+
 def test_static_scratch_reports_through_status_word():
     """A bad page-table entry is reported in the caller's status word, sticky, and
     cleared by writing 0."""
