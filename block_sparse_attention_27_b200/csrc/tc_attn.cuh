@@ -219,6 +219,42 @@ struct Engine {
   // Runs the pipeline over `num_tiles` tiles.  Softmax threads return their
   // row's (m, l) in the log2 domain (l over both halves) and whether the CTA is
   // still alive.
+  //
+  // Phase accounting.  A parity wait on an mbarrier tells apart only two
+  // consecutive phases, so every wait below is made while the barrier has
+  // completed either the phase before the one waited for or that phase itself:
+  // never two behind (the wait would return at once) and never one past (it
+  // would block until the timeout).  For each barrier: who completes it, who
+  // waits for which completion, and why the completion after it cannot have
+  // happened yet; the one before it always has, because each waiter waited for
+  // it (or for a later event that follows it) on its previous use.  This holds
+  // for any STAGES >= 3 with kLook = 2; with STAGES = 2, kLook = 1 and the same
+  // arguments hold one tile closer.
+  //   kv_full(st)  TMA of tile k (the (k / STAGES)-th fill of stage st).  The MMA
+  //                issuer (S(k)) and softmax thread r (value-row zeroing) wait
+  //                for it; the next fill of st is tile k + STAGES, issued after
+  //                kv_empty(st) of PV(k), which follows both waits.
+  //   kv_empty(st) commit after PV(j), j % STAGES == st; the producer waits for
+  //                PV(k - STAGES) before it loads tile k into st; the next commit,
+  //                PV(k), needs tile k loaded.
+  //   s_full(sb)   commit of S(k) into buffer s_buf(k); softmax group k % 2 waits
+  //                for it as its (mine / 2)-th use of sb; S(k + 4) into sb needs
+  //                s_free(sb) from this very read.
+  //   s_free(sb)   128 softmax arrivals once S(k) is read; the issuer waits for
+  //                the one of tile k - 4 before S(k); the next (tile k) needs S(k).
+  //   p_full(g, m & 1)  128 arrivals once P of group g's m-th tile is in TMEM, two
+  //                barriers used alternately; the issuer waits for it before
+  //                PV; the next arrival on the same barrier is for m + 2, whose S
+  //                the issuer sends only after this wait.
+  //   pv_done(g)   commit after each PV of group g.  The issuer waits, before
+  //                S(k) overwrites the TMEM buffer that held P(k - 4), for
+  //                PV(k - 4): at that point it has issued PVs up to k - 3, so
+  //                PV(k - 4) is the latest of its group.  Softmax group g waits,
+  //                before rescaling O for its m-th tile, for the PV of its
+  //                (m - 1)-th; PV of the m-th needs this group's P first, and PV
+  //                of the (m - 2)-th completed before S of the m-th was issued.
+  //   drain        one commit after the issuer's last MMA; a one-phase barrier,
+  //                waited for once by every softmax thread before O is read.
   template <int PAGE, class Policy>
   __device__ __forceinline__ bool run(Policy &pol, int num_tiles, float &m_out, float &l_out) {
     using namespace sm100;
