@@ -51,7 +51,7 @@ struct PartialParams {
 // and that max (mtile); the split's unnormalised O row, m and l go to part_o /
 // part_ml.
 // ---------------------------------------------------------------------------
-constexpr int kSelStages = 5;
+constexpr int kSelStages = 6;  // three pairs of stages (the engine's PAIR mode)
 
 // K/V tiles are read once: loaded with an evict-first L2 policy, so that the
 // partials the tail reads back (written during the loop) stay in L2.
@@ -856,7 +856,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   pol.vmap = &vmap;
   pol.kmap4 = &kmap4;
   pol.vmap4 = &vmap4;
-  tc::Engine<D, kSelStages> eng;
+  tc::Engine<D, kSelStages, true> eng;
   eng.setup(smem_raw, pol);
   // everything below may read what the kernel ahead of this one wrote
   sm100::grid_dep_wait();

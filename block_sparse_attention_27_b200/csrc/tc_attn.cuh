@@ -8,7 +8,11 @@
 //               instruction per tile) into a STAGES-deep ring of
 //               128-byte-swizzled shared tiles;
 //   warp 1      TMEM owner and MMA issuer: S_k = Q K_k^T into a double-buffered
-//               TMEM S (64 fp32 columns each), O += P_k V_k into TMEM O;
+//               TMEM S (64 fp32 columns each), O += P_k V_k into TMEM O.  With
+//               PAIR, the S of tiles 2m and 2m + 1 is one MMA chain of N = 128
+//               (their K tiles sit in adjacent stages, their S buffers in
+//               adjacent TMEM columns): half the S instructions, and the Q
+//               operand is read from shared memory once per two tiles;
 //   warps 2..9  two softmax warpgroups that take alternate tiles (group g
 //               the tiles k with k % 2 == g), so that one group's exp phase
 //               overlaps the other's loads and stores.  Thread (g, r) owns query
@@ -72,9 +76,15 @@ struct Layout {
   static_assert(D == 64 || D == 128, "head dimension");
 };
 
-template <int D, int STAGES>
+template <int D, int STAGES, bool PAIR = false>
 struct Engine {
   using L = Layout<D, STAGES>;
+  static_assert(!PAIR || (STAGES % 2 == 0 && STAGES >= 4), "tile pairs fill adjacent stages");
+  // Distance between the two 64-element halves of a K or V tile in shared
+  // memory.  With PAIR a pair of stages is [K half 0: tile 2m, tile 2m + 1][K
+  // half 1: ...][V half 0: ...][V half 1: ...], so that the K rows of both tiles
+  // of a half are one 128-row operand.
+  static constexpr uint32_t kHalfStride = PAIR ? 2 * L::kKVHalf : L::kKVHalf;
   uint32_t base;         // 1 KB-aligned shared address of the layout
   unsigned char *smem;   // same, generic pointer
   uint32_t tmem;         // TMEM base address (lane 0, column 0)
@@ -96,10 +106,20 @@ struct Engine {
   __device__ __forceinline__ uint32_t drain() const { return bar(2 * STAGES + 15); }
   __device__ __forceinline__ uint32_t user_bar() const { return bar(2 * STAGES + 16); }
   // tile k runs on softmax group k % 2 as that group's (k / 2)-th tile, in S buffer
-  // 2 * group + (k / 2) % 2
-  static __device__ __forceinline__ int s_buf(int k) { return 2 * (k & 1) + ((k >> 1) & 1); }
-  __device__ __forceinline__ uint32_t stage_k(int st) const { return base + L::kOffKV + st * L::kStageBytes; }
-  __device__ __forceinline__ uint32_t stage_v(int st) const { return stage_k(st) + L::kKBytes; }
+  // 2 * group + (k / 2) % 2; with PAIR in buffer 2 * ((k / 2) % 2) + group, so
+  // that the two tiles of a pair have adjacent buffers.  Either way a group's
+  // tiles alternate between its two buffers.
+  static __device__ __forceinline__ int s_buf(int k) {
+    return PAIR ? 2 * ((k >> 1) & 1) + (k & 1) : 2 * (k & 1) + ((k >> 1) & 1);
+  }
+  // half 0 of stage st's K and V tiles (half 1 is kHalfStride further)
+  __device__ __forceinline__ uint32_t stage_k(int st) const {
+    return PAIR ? base + L::kOffKV + (st >> 1) * 2 * L::kStageBytes + (st & 1) * L::kKVHalf
+                : base + L::kOffKV + st * L::kStageBytes;
+  }
+  __device__ __forceinline__ uint32_t stage_v(int st) const {
+    return stage_k(st) + (PAIR ? 2 * L::kKBytes : L::kKBytes);
+  }
   __device__ __forceinline__ volatile int *abort_flag() const {
     return reinterpret_cast<volatile int *>(smem + L::kOffMisc + 4);
   }
@@ -212,7 +232,7 @@ struct Engine {
   __device__ __forceinline__ void issue_first(Policy &pol, int num_tiles) {
     if (lane == 0) DSA_TRACE_EVENT(36);
     for (int k = 0; k < min(STAGES, num_tiles); ++k)
-      pol.load_tile(k, stage_k(k), stage_v(k), L::kKVHalf, kv_full(k), lane);
+      pol.load_tile(k, stage_k(k), stage_v(k), kHalfStride, kv_full(k), lane);
     if (lane == 0) DSA_TRACE_EVENT(2);
   }
 
@@ -253,6 +273,9 @@ struct Engine {
   //                before rescaling O for its m-th tile, for the PV of its
   //                (m - 1)-th; PV of the m-th needs this group's P first, and PV
   //                of the (m - 2)-th completed before S of the m-th was issued.
+  //                With PAIR, pair m + 1 (tiles k = 2m + 2 and 2m + 3) waits at
+  //                the top of iteration 2m, when PVs up to 2m - 1 are out:
+  //                PV(k - 4) is again the latest of tile k's group.
   //   drain        one commit after the issuer's last MMA; a one-phase barrier,
   //                waited for once by every softmax thread before O is read.
   template <int PAGE, class Policy>
@@ -271,7 +294,7 @@ struct Engine {
         for (int k = issued; k < num_tiles; ++k) {
           const int st = k % STAGES;
           if (!__all_sync(0xffffffffu, mbar_wait(kv_empty(st), ((k / STAGES) - 1) & 1, ctx))) break;
-          pol.load_tile(k, stage_k(st), stage_v(st), L::kKVHalf, kv_full(st), lane);
+          pol.load_tile(k, stage_k(st), stage_v(st), kHalfStride, kv_full(st), lane);
           if (k == STAGES && lane == 0) DSA_TRACE_EVENT(24);
           issued = k + 1;
         }
@@ -307,7 +330,7 @@ struct Engine {
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t hf = kk >> 2, sub = kk & 3;
             const uint64_t ad = sdesc_sw128(base + L::kOffQ + hf * L::kQHalf + sub * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sk + hf * L::kKVHalf + sub * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sk + hf * kHalfStride + sub * 32, 16, 1024);
             umma_bf16(tmem + sb * kBN, ad, bd, kIdS, kk > 0 ? 1u : 0u);
           }
           umma_commit(s_full(sb));
@@ -315,11 +338,54 @@ struct Engine {
           if (k == 4) DSA_TRACE_EVENT(15);
           return true;
         };
+        // PAIR: S of tiles 2m and 2m + 1 (of tile 2m alone when it is the last)
+        // as one chain of N = 2 kBN into their adjacent buffers.  Pair m + 1 is
+        // issued at the top of iteration 2m, after the PVs up to 2m - 1, so that
+        // the PV(k - 4) it waits for is the latest PV of tile k's group.  (Sent
+        // instead after PV(2m), it leaves group 0 without an S for the length
+        // of PV(2m) and the pair's MMAs: a slower loop, although that needs no
+        // wait for a PV just issued.)
+        constexpr uint32_t kIdS2 = idesc_bf16(128, 2 * kBN, false, false);
+        auto issue_pair = [&](int m) -> bool {
+          const int k0 = 2 * m;
+          const int nk = k0 + 1 < num_tiles ? 2 : 1;
+          for (int t = 0; t < nk; ++t) {
+            const int k = k0 + t;
+            if (!mbar_wait(kv_full(k % STAGES), (k / STAGES) & 1, ctx)) return false;
+            if (k >= 4) {
+              if (!mbar_wait(s_free(s_buf(k)), (((k >> 1) - 2) >> 1) & 1, ctx)) return false;
+              if (!mbar_wait(pv_done(k & 1), ((k >> 1) - 2) & 1, ctx)) return false;
+            }
+          }
+          if (k0 == 0) DSA_TRACE_EVENT(3);
+          tc_fence_after();
+          const uint32_t sk = stage_k(k0 % STAGES);  // tile k0's rows, then tile k0 + 1's
+          const uint32_t dst = tmem + s_buf(k0) * kBN;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t hf = kk >> 2, sub = kk & 3;
+            const uint64_t ad = sdesc_sw128(base + L::kOffQ + hf * L::kQHalf + sub * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sk + hf * kHalfStride + sub * 32, 16, 1024);
+            umma_bf16(dst, ad, bd, nk == 2 ? kIdS2 : kIdS, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full(s_buf(k0)));
+          if (nk == 2) umma_commit(s_full(s_buf(k0 + 1)));
+          return true;
+        };
         bool ok = mbar_wait(q_full(), 0, ctx);
         DSA_TRACE_EVENT(12);
-        for (int k = 0; ok && k < kLook && k < num_tiles; ++k) ok = issue_s(k);
+        if constexpr (PAIR) {
+          if (ok) ok = issue_pair(0);
+          if (ok && num_tiles > 2) ok = issue_pair(1);
+        } else {
+          for (int k = 0; ok && k < kLook && k < num_tiles; ++k) ok = issue_s(k);
+        }
         for (int j = 0; ok && j < num_tiles; ++j) {
-          if (j + kLook < num_tiles && !issue_s(j + kLook)) break;
+          if constexpr (PAIR) {
+            if ((j & 1) == 0 && j >= 2 && j + 2 < num_tiles && !issue_pair((j >> 1) + 1)) break;
+          } else {
+            if (j + kLook < num_tiles && !issue_s(j + kLook)) break;
+          }
           const int st = j % STAGES, g = j & 1;
           if (!mbar_wait(p_full(g, j >> 1), (j >> 2) & 1, ctx)) break;
           if (j == 2) DSA_TRACE_EVENT(14);
@@ -328,7 +394,7 @@ struct Engine {
           const uint32_t pa = tmem + s_buf(j) * kBN;  // P_j in TMEM: 8 columns per 16 keys
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t bd = sdesc_sw128(sv + kk * 16 * 128, L::kKVHalf, 1024);
+            const uint64_t bd = sdesc_sw128(sv + kk * 16 * 128, kHalfStride, 1024);
             umma_bf16_ts(tmem + L::kTmemO + g * D, pa + kk * 8, bd, kIdO, (j > 1 || kk > 0) ? 1u : 0u);
           }
           umma_commit(pv_done(g));
@@ -437,7 +503,7 @@ struct Engine {
           for (int hf = 0; hf < L::kHalves; ++hf)
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4 *>(vrow + hf * L::kKVHalf + c * 16) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4 *>(vrow + hf * kHalfStride + c * 16) = make_uint4(0, 0, 0, 0);
         }
         pol.after_tile(k, r, m_used, usum);
         if (tr) DSA_TRACE_EVENT(22);
