@@ -1150,49 +1150,56 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // ---------------------------------------------------------------------------
 // Calls f(key, position) for every (KV head, page) pair of a sequence, position
 // h * np + q; rows of the score array are max_pages apart.  16-byte loads, eight
-// per thread in flight, when the rows are 16-byte aligned.
+// per thread in flight, when the rows are 16-byte aligned.  A flat index v over
+// rows of n items splits as (h, j) = (v / n, v % n) with one division per eight
+// items: the next item of the thread is nt further, i.e. nt / n rows and nt % n
+// items on.
 template <class F>
 __device__ __forceinline__ void for_each_pair(const float *scores, int max_pages, int Hkv, int np, F f) {
   const int nt = (int)blockDim.x;
-  if ((max_pages & 3) == 0) {
-    const int nv = (np + 3) >> 2, tot = Hkv * nv;
-    for (int v0 = threadIdx.x; v0 < tot; v0 += 8 * nt) {
-      float4 x[8];
+  const bool vec = (max_pages & 3) == 0;
+  const int n = vec ? (np + 3) >> 2 : np;  // items per row: 4-page vectors or pages
+  const int tot = Hkv * n;
+  if (tot <= 0) return;
+  const int dq = nt / n, dr = nt - dq * n;
+  for (int v0 = threadIdx.x; v0 < tot; v0 += 8 * nt) {
+    int hh[8], jj[8];
+    {
+      int h = v0 / n, j = v0 - h * n;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int v = v0 + u * nt;
-        if (v < tot) {
-          const int h = v / nv, j = v - h * nv;
-          x[u] = __ldcg(reinterpret_cast<const float4 *>(scores + (size_t)h * max_pages) + j);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int v = v0 + u * nt;
-        if (v < tot) {
-          const int h = v / nv, j = v - h * nv;
-          const float e[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            if (4 * j + c < np) f(score_key(e[c]), h * np + 4 * j + c);
+        hh[u] = h;
+        jj[u] = j;
+        h += dq;
+        j += dr;
+        if (j >= n) {
+          j -= n;
+          ++h;
         }
       }
     }
-  } else {
-    const int tot = Hkv * np;
-    for (int i0 = threadIdx.x; i0 < tot; i0 += 8 * nt) {
-      float x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * nt;
-        if (i < tot) {
-          const int h = i / np;
-          x[u] = __ldcg(scores + (size_t)h * max_pages + (i - h * np));
-        }
-      }
+    if (vec) {
+      float4 x[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
-        if (i0 + u * nt < tot) f(score_key(x[u]), i0 + u * nt);
+        if (hh[u] < Hkv) x[u] = __ldcg(reinterpret_cast<const float4 *>(scores + (size_t)hh[u] * max_pages) + jj[u]);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (hh[u] < Hkv) {
+          const float e[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (4 * jj[u] + c < np) f(score_key(e[c]), hh[u] * np + 4 * jj[u] + c);
+        }
+      }
+    } else {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (hh[u] < Hkv) x[u] = __ldcg(scores + (size_t)hh[u] * max_pages + jj[u]);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (hh[u] < Hkv) f(score_key(x[u]), hh[u] * np + jj[u]);
     }
   }
 }
@@ -1250,8 +1257,9 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
   uint32_t t0 = 0u;  // candidates: every key >= t0
   if (fast) {
     // 1. the key range holding the take-th largest key: the range of all keys
-    //    (one pass), then histograms of 4096 equal bins over the current range,
-    //    narrowed to the bin that holds it while that bin has too many keys
+    //    (one pass), then histograms of up to 4096 bins of 2^shift keys over the
+    //    current range, narrowed to the bin that holds it while that bin has
+    //    too many keys
     uint32_t kmn = 0xffffffffu, kmx = 0u;
     for_each_pair(scores, sh.max_pages, sh.Hkv, np, [&](uint32_t key, int) {
       kmn = min(kmn, key);
@@ -1275,7 +1283,9 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
     __syncthreads();  // (sc is reused)
     uint32_t above = 0u;  // keys above the current range
     for (int level = 0; level < 4; ++level) {
-      const uint32_t width = (uint32_t)(((unsigned long long)(hi - lo) + kHist) / kHist);  // >= 1
+      uint32_t shift = 0u;  // the smallest with (hi - lo) >> shift < kHist
+      while (((hi - lo) >> shift) >= (uint32_t)kHist) ++shift;
+      const uint32_t width = 1u << shift;
       for (int i = tid; i < kHist; i += nt) hist[i] = 0u;
       if (tid == 0) {
         s_bin = 0u;
@@ -1283,7 +1293,7 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
       }
       __syncthreads();
       for_each_pair(scores, sh.max_pages, sh.Hkv, np, [&](uint32_t key, int) {
-        if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) / width], 1u);
+        if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) >> shift], 1u);
       });
       __syncthreads();
       // the bin of the take-th largest key: warp 0 scans from the top
