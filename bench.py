@@ -639,11 +639,11 @@ def _run_ours(args, world, rank, local, dsa):
 
     # the other workloads, timed the same way (each its own graphs over its own
     # layer copies; the batched workload holds ~1.3 GB of cache per layer, so fewer)
-    configs = {}
+    others = {}
     for name in [c for c in args.configs.split(",") if c and c != "none" and c != args.workload]:
         wc = W.make(name, 0)
         mc = measure(wc, LAYERS.get(name, 64), dsa, args.steps, args.warmup, world, args.select_sms)
-        configs[name] = config_entry(wc, mc, LAYERS.get(name, 64), hbm_peak, world,
+        others[name] = config_entry(wc, mc, LAYERS.get(name, 64), hbm_peak, world,
                                      cpu=(world == 1 and not args.no_cpu_baseline))
         del mc, wc
         torch.cuda.empty_cache()
@@ -722,7 +722,7 @@ def _run_ours(args, world, rank, local, dsa):
                                      "of sparse over exact attention at every step; eager launches",
                              **shape},
     }
-    line["configs"] = configs
+    line["configs"] = others
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line, ensure_ascii=False), flush=True)
