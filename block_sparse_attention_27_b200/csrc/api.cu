@@ -220,6 +220,8 @@ int dsa_select(const void *q_blk, const void *k_cache, const void *v_cache,
   a.scores = at<float>(workspace, plan.off_scores);
   a.cand = at<uint64_t>(workspace, plan.off_cand);
   a.ccnt = at<int32_t>(workspace, plan.off_ccnt);
+  a.hsel = at<int32_t>(workspace, plan.off_hsel);
+  a.hcnt = at<int32_t>(workspace, plan.off_hcnt);
   a.counters = at<uint32_t>(workspace, plan.off_counters);
   a.status = at<uint32_t>(workspace, 0);
   if (dsa::launch_select(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -261,6 +263,8 @@ int dsa_select_static_scratch(const void *q_blk, const void *k_cache, const void
   a.scores = at<float>(scratch, plan.off_scores);
   a.cand = at<uint64_t>(scratch, plan.off_cand);
   a.ccnt = at<int32_t>(scratch, plan.off_ccnt);
+  a.hsel = at<int32_t>(scratch, plan.off_hsel);
+  a.hcnt = at<int32_t>(scratch, plan.off_hcnt);
   a.counters = at<uint32_t>(scratch, plan.off_counters);
   a.status = status;  // the caller's word; the array's header holds only the group counters
   if (dsa::launch_select(sh, plan, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -72,7 +72,8 @@ struct SelectPlan {
   int bgp;               // BG rounded up to a multiple of 4: row stride of pagepart / mtile
   int slot_len;          // entries of one CTA's candidate list
   size_t off_counters;   // in the zeroed header: four counters per group of a launch
-  size_t off_part_o, off_part_ml, off_pagepart, off_mtile, off_scores, off_cand, off_ccnt, total;
+  size_t off_part_o, off_part_ml, off_pagepart, off_mtile, off_scores, off_cand, off_ccnt, off_hsel,
+      off_hcnt, total;
 };
 
 // Counters of a group (barrier arrivals, candidate hand-offs, output rows taken,
@@ -92,6 +93,8 @@ struct SelectArgs {
   float *scores;      // [S*Hkv][max_pages]
   uint64_t *cand;     // [S*Hkv][group_ctas][slot_len] local candidates (score bits << 32 | ~page)
   int32_t *ccnt;      // [S*Hkv][group_ctas] candidates of each CTA
+  int32_t *hsel;      // [S*Hkv][max_pages] head-adaptive budget: each head's best pages
+  int32_t *hcnt;      // [S*Hkv] their number
   uint32_t *counters; // [groups_per_launch][4] (arrive, leave, output rows, done)
   uint32_t *status;
 };

@@ -993,18 +993,22 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
   __syncthreads();
 
   // ---- 3. row statistics, page scores, local candidates ----
-  // (under the head-adaptive budget the selection is select_global_topk's: this
-  // kernel only writes the page scores)
+  // Under the head-adaptive budget the final selection is select_global_topk's:
+  // this kernel writes the page scores and each head's best kh = min(Hkv kp, np)
+  // pages, which hold every page of the head that the shared budget of Hkv kp
+  // keeps (within a head the two rankings agree, so a kept page has fewer than
+  // Hkv kp pages of its own head above it).
   const bool per_head = sh.head_budget == 0;
   int kp = topk_tokens / PAGE;
   if ((per_head && kp > sh.kmax) || kp < 0 || topk_tokens % PAGE != 0) {
     if (threadIdx.x == 0 && c == 0) raise_status(a.status, kStatusBadIndex);
     kp = max(0, min(kp, sh.kmax));
   }
-  const int take = min(kp, np);
-  const bool every_page = take >= np || !per_head;
-  const bool fast = kp <= kFastTopk;
-  const int E = every_page ? 0 : (!fast ? 0 : (kp <= 32 ? 1 : (kp <= 64 ? 2 : 4)));
+  const int kh = per_head ? kp : (int)min((long long)sh.Hkv * kp, (long long)np);
+  const int take = min(kh, np);
+  const bool every_page = take >= np;
+  const bool fast = kh <= kFastTopk;
+  const int E = every_page ? 0 : (!fast ? 0 : (kh <= 32 ? 1 : (kh <= 64 ? 2 : 4)));
   merged_row_stats(sh, plan, a.part_ml, sh_idx, sM, sLinv, [&]() {
     if (threadIdx.x == 0 && !started) st.start();
   });
@@ -1048,15 +1052,18 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
     if (sc.flag) __threadfence();  // the other CTAs' candidates are visible from here on
   }
   __syncthreads();
-  if (sc.flag && per_head) {
-    int32_t *out = a.idx_out + sh_idx * sh.kmax;
+  if (sc.flag) {
+    // per head: idx_out, padded with -1 to kmax; head-adaptive budget: the head's
+    // list for select_global_topk, take entries
+    int32_t *out = per_head ? a.idx_out + sh_idx * sh.kmax : a.hsel + sh_idx * sh.max_pages;
+    const int out_len = per_head ? sh.kmax : take;
     const uint64_t *lists = a.cand + sh_idx * G * plan.slot_len;
     if (every_page) {
-      for (int i = threadIdx.x; i < sh.kmax; i += blockDim.x) out[i] = i < np ? i : -1;
+      for (int i = threadIdx.x; i < out_len; i += blockDim.x) out[i] = i < np ? i : -1;
     } else if (fast) {
-      if (E == 1) final_topk_fast<1>(lists, plan.slot_len, G, take, out, sh.kmax, wl);
-      else if (E == 2) final_topk_fast<2>(lists, plan.slot_len, G, take, out, sh.kmax, wl);
-      else final_topk_fast<4>(lists, plan.slot_len, G, take, out, sh.kmax, wl);
+      if (E == 1) final_topk_fast<1>(lists, plan.slot_len, G, take, out, out_len, wl);
+      else if (E == 2) final_topk_fast<2>(lists, plan.slot_len, G, take, out, out_len, wl);
+      else final_topk_fast<4>(lists, plan.slot_len, G, take, out, out_len, wl);
     } else {
       // offsets of the CTAs' candidate lists (CTA order is page order)
       int *offs = reinterpret_cast<int *>(tail + kTailHead);
@@ -1067,7 +1074,7 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
       if (warp == 0) {
         int carry = 0;
         for (int j0 = 0; j0 < G; j0 += 32) {
-          const int v = j0 + lane < G ? min(max(__ldcg(a.ccnt + sh_idx * G + j0 + lane), 0), sh.kmax) : 0;
+          const int v = j0 + lane < G ? min(max(__ldcg(a.ccnt + sh_idx * G + j0 + lane), 0), plan.slot_len) : 0;
           int incl = v;
 #pragma unroll
           for (int o = 1; o < 32; o <<= 1) {
@@ -1095,10 +1102,11 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
         block_topk(np, take, [&](int i) -> uint32_t { return score_key(__ldcg(gs + i)); },
                    [&](int i, int pos) { out[pos] = i; }, sc);
       }
-      for (int i = take + threadIdx.x; i < sh.kmax; i += blockDim.x) out[i] = -1;
+      for (int i = take + threadIdx.x; i < out_len; i += blockDim.x) out[i] = -1;
     }
     if (threadIdx.x == 0) {
-      a.cnt_out[sh_idx] = take;
+      if (per_head) a.cnt_out[sh_idx] = take;
+      else a.hcnt[sh_idx] = take;
       DSA_TRACE_EVENT(43);
     }
   }
@@ -1255,7 +1263,12 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
   constexpr int kHist = kGlobalHistBins;
   bool fast = total <= kGlobalBits && take > 0 && take < total;
   uint32_t t0 = 0u;  // candidates: every key >= t0
-  if (fast) {
+  // the candidates can be the heads' lists of select_fused (each head's best
+  // min(Hkv kp, np) pages, which hold every pair the budget keeps) when they fit
+  int ncl = 0;
+  for (int h = 0; h < sh.Hkv; ++h) ncl += min(max(a.hcnt[(size_t)s * sh.Hkv + h], 0), np);
+  const bool from_lists = fast && ncl <= kGlobalCand;
+  if (fast && !from_lists) {
     // 1. the key range holding the take-th largest key: the range of all keys
     //    (one pass), then histograms of up to 4096 bins of 2^shift keys over the
     //    current range, narrowed to the bin that holds it while that bin has
@@ -1333,15 +1346,34 @@ __global__ void __launch_bounds__(kGlobalThreads) select_global_topk(const __gri
     fast = s_above <= (uint32_t)kGlobalCand;
   }
   if (fast) {
-    // 2. candidates: every key >= t0, with its position
-    if (tid == 0) s_ncand = 0u;
+    // 2. candidates with their positions: the heads' lists, or every key >= t0
+    if (tid == 0) s_ncand = from_lists ? (uint32_t)ncl : 0u;
     __syncthreads();
-    for_each_pair(scores, sh.max_pages, sh.Hkv, np, [&](uint32_t key, int pos) {
-      if (key >= t0) {
-        const uint32_t slot = atomicAdd(&s_ncand, 1u);
-        if (slot < (uint32_t)kGlobalCand) cand[slot] = make_uint2(key, (uint32_t)pos);
+    if (from_lists) {
+      for (int i = tid; i < ncl; i += nt) {
+        int h = 0, base = 0;
+        for (;;) {  // the head whose list holds entry i (ncl counts every list)
+          const int c = min(max(a.hcnt[(size_t)s * sh.Hkv + h], 0), np);
+          if (i < base + c || h == sh.Hkv - 1) break;
+          base += c;
+          ++h;
+        }
+        int page = a.hsel[((size_t)s * sh.Hkv + h) * sh.max_pages + (i - base)];
+        if (page < 0 || page >= np) {
+          raise_status(a.status, kStatusBadIndex);
+          page = 0;
+        }
+        cand[i] = make_uint2(score_key(__ldcg(scores + (size_t)h * sh.max_pages + page)),
+                             (uint32_t)(h * np + page));
       }
-    });
+    } else {
+      for_each_pair(scores, sh.max_pages, sh.Hkv, np, [&](uint32_t key, int pos) {
+        if (key >= t0) {
+          const uint32_t slot = atomicAdd(&s_ncand, 1u);
+          if (slot < (uint32_t)kGlobalCand) cand[slot] = make_uint2(key, (uint32_t)pos);
+        }
+      });
+    }
     for (int w = tid; w < (total + 31) / 32; w += nt) {
       keep[w] = 0u;
       eqb[w] = 0u;
@@ -1570,6 +1602,10 @@ SelectPlan plan_select(const Shape &sh, int num_sms) {
   } else {
     p.slot_len = sh.kmax;
   }
+  // head-adaptive budget: a CTA's list holds up to 128 keys (kh <= 128) or up to
+  // the pages of its split (kh > 128), whatever kmax is
+  if (sh.head_budget)
+    p.slot_len = std::max(p.slot_len, std::max(kFastTopk, p.tiles_per_split * (tc::kBN / std::min(sh.P, tc::kBN))));
   // groups of one launch: all of their CTAs resident at once
   p.group_ctas = p.splits * p.rowtiles;
   p.groups_per_launch = (int)std::max(1LL, std::min<long long>(kMaxGroupsPerLaunch, num_sms / p.group_ctas));
@@ -1588,6 +1624,8 @@ SelectPlan plan_select(const Shape &sh, int num_sms) {
   p.off_scores = off;   off = align(off + shn * sh.max_pages * 4);
   p.off_cand = off;     off = align(off + shn * p.group_ctas * p.slot_len * 8);
   p.off_ccnt = off;     off = align(off + shn * p.group_ctas * 4);
+  p.off_hsel = off;     off = align(off + shn * sh.max_pages * 4);
+  p.off_hcnt = off;     off = align(off + shn * 4);
   p.total = off;
   return p;
 }
