@@ -417,6 +417,28 @@ def pin_global_concentrated_head(orc):
     assert r.cnt[0, 1] == w.Hkv * w.kmax - len(pages)
 
 
+def pin_global_within_head_lists(orc):
+    """Every (head, page) pair the shared budget keeps is among its own head's best
+    min(Hkv kp, np) pages by the per-head rule: within one head both rankings order
+    pages by score, then lower page.  (A two-step selection, per head first, rests on
+    this.)  Ragged paged sequences, three heads, and all-equal scores (zero keys, so
+    every full page ties and the tie rules alone decide)."""
+    zero = brute_sized(8, n=180, topk=32, Hkv=2, Hq=4, needle_count=0)
+    zero = W.Workload(**{**zero.__dict__, "k_cache": torch.zeros_like(zero.k_cache)})
+    for w in (small_paged(5), brute_sized(4, Hkv=3, Hq=6, topk=16), zero):
+        g = run_global(orc, w)
+        cap = torch.tensor([w.n_pages(s) * w.P for s in range(w.S)], dtype=torch.int32)
+        wide = W.Workload(**{**w.__dict__, "topk": torch.minimum(w.topk * w.Hkv, cap)})
+        r = run(orc, wide, kmax=w.max_pages)
+        for s in range(w.S):
+            for h in range(w.Hkv):
+                kept = set(g.idx[s, h, :g.cnt[s, h]].tolist())
+                best = set(r.idx[s, h, :r.cnt[s, h]].tolist())
+                assert kept <= best, (s, h, sorted(kept - best))
+            assert sum(int(g.cnt[s, h]) for h in range(w.Hkv)) == min(
+                w.Hkv * int(w.topk[s]) // w.P, w.Hkv * w.n_pages(s))
+
+
 # ---------------------------------------------------------- LoSA prefix reuse
 def run_losa(orc, w, idx, cnt, active, cache_o, cache_lse, q=None, bk=None, bv=None):
     return orc.sparse_losa(W.bits(w.q1 if q is None else q), W.bits(w.k_cache), W.bits(w.v_cache),
@@ -487,4 +509,4 @@ FAST_PINS = [pin_score_sums, pin_dense_equivalence, pin_topk_brute_force,
              pin_query_order_invariance, pin_single_row, pin_budget_covers_prefix,
              pin_ascending_and_padding, pin_worked_example, pin_rejects_bad_indices,
              pin_global_brute_force, pin_global_one_head_is_per_head, pin_global_covers_prefix,
-             pin_global_concentrated_head, pin_losa]
+             pin_global_concentrated_head, pin_global_within_head_lists, pin_losa]
