@@ -21,8 +21,9 @@
 //      top-kp of its own CTA) and writes them ascending.
 //   5. Every CTA merges rows of o_out = sum_j 2^(m_j - M) O_j / L, taken from
 //      a counter.
-// select_global_topk (head-adaptive budget only) then selects over all KV
-// heads of each sequence, from the page scores select_fused wrote.
+// Under the head-adaptive budget steps 3-4 keep kh = min(Hkv kp, np) pages per
+// head instead, into a workspace list, and select_global_topk then selects over
+// all KV heads of each sequence from those lists.
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -1143,13 +1144,14 @@ __global__ void __launch_bounds__(tc::kThreads, 1)
 // ascending order, a head keeping any number of them (none included).
 //
 // Fast path (positions <= kGlobalBits, candidates <= kGlobalCand):
-//   1. the range of the keys (one pass, coalesced 16-byte loads), then a
-//      histogram of 4096 equal bins over it gives the bin holding the
-//      take-th largest key; while that bin holds too many keys, a histogram
-//      over the bin narrows it; t0 = the lower edge of the bin found;
-//   2. the keys >= t0 are compacted into shared memory with their positions,
-//      and an exact radix select among them gives T and the number of keys == T
-//      to keep;
+//   1. the candidates: the heads' lists of select_fused (each head's best
+//      min(Hkv kp, np) pages, which hold every kept pair) when they number at
+//      most kGlobalCand; otherwise the range of all keys (one pass, coalesced
+//      16-byte loads), then histograms of up to 4096 bins over it give the bin
+//      holding the take-th largest key, narrowed while it holds too many keys,
+//      and the keys >= its lower edge t0 are compacted;
+//   2. with their positions in shared memory, an exact radix select among the
+//      candidates gives T and the number of keys == T to keep;
 //   3. bitmaps over the positions: keys > T kept, keys == T kept in ascending
 //      position until need_eq of them;
 //   4. warp h writes head h's kept pages (its stretch of the bitmap) in order.
