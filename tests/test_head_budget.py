@@ -94,17 +94,28 @@ def test_head_budget_launches(dsa_mod):
     assert dsa_mod.select_launches(dw1.dims) == 1
 
 
-@pytest.mark.parametrize("n,Hkv,path", [(1000, 2, "staged candidates"), (20000, 8, "keys from L2")])
-def test_head_budget_all_ties(dsa_mod, n, Hkv, path):
+@pytest.mark.parametrize("n,Hkv,topk,path", [(1000, 2, 256, "head lists"), (20000, 8, 256, "head lists"),
+                                              (40000, 8, 4096, "every pair, keys from L2")])
+def test_head_budget_all_ties(dsa_mod, n, Hkv, topk, path):
     """All keys zero: every full page of every head has the same score, bit for bit,
     on both sides.  The shared budget then goes to the lowest (head, page) pairs:
     head 0 takes it all and the other heads keep nothing (the sparse pass then
-    attends to the block alone for them).  Covers both selection paths."""
-    w = W.make("tiny", 3, n=n, topk=256, B=4, Hq=2 * Hkv, Hkv=Hkv, d=64, needle_count=0)
+    attends to the block alone for them).  The last case's head lists (8 x 2048)
+    exceed the global kernel's staging area, so it ranks every pair, and with all
+    keys equal no histogram narrows them: its radix passes read the keys from L2."""
+    w = W.make("tiny", 3, n=n, topk=topk, B=4, Hq=2 * Hkv, Hkv=Hkv, d=64, needle_count=0)
     w.k_cache = torch.zeros_like(w.k_cache)
     dw, ref = run_global_case(dsa_mod, w)
     got = dw.idx.cpu().numpy()
-    K = Hkv * (256 // w.P)
+    K = Hkv * (topk // w.P)
     assert int(dw.cnt[0, 0]) == K and got[0, 0, :K].tolist() == list(range(K))
     assert dw.cnt[0, 1:].sum().item() == 0
     assert np.array_equal(got, ref.idx) and np.array_equal(dw.cnt.cpu().numpy(), ref.cnt)
+
+
+def test_head_budget_long_lists(dsa_mod):
+    """Head lists longer than the global kernel's staging area (8 x 2048 > 8192
+    candidates): it ranks every (head, page) pair instead, through the key range,
+    histogram narrowing and compaction of the keys above the cut."""
+    run_global_case(dsa_mod, W.make("tiny", 5, n=40000, topk=4096, B=4, Hq=16, Hkv=8, d=64,
+                                    needle_count=16))
