@@ -161,11 +161,13 @@ typedef struct CUstream_st *dsa_stream_t;
  * [S]); page (must equal dims->page); topk (DEVICE int32 [S], tokens); idx_out
  * (device int32 [S,Hkv,kmax]); o_out (device bf16 [S,B,Hq,d]); stream; dims;
  * cnt_out (device int32 [S,Hkv]); workspace/ws_bytes (device, see above).
- * Launches: one cooperative kernel per dsa_select_launches(dims) groups of
- * (sequence, KV head) whose CTAs are all resident at once (one launch when
- * S * Hkv * ceil(B * Hq/Hkv / 128) does not exceed the SMs it may use).  The
- * CTAs of a (sequence, KV head) wait for one another at one point, with a
- * bounded wait (DSA_ERR_DEVICE_TIMEOUT if it gives up).
+ * Launches: dsa_select_launches(dims) kernels in all: the selection kernel once
+ * per batch of (sequence, KV head) groups whose CTAs are all resident at once
+ * (one batch when S * Hkv * ceil(B * Hq/Hkv / 128) does not exceed the SMs it may
+ * use), each group a thread-block cluster when it has at most 16 CTAs, else the
+ * batch one cooperative launch; with head_budget = 1, one more kernel for the
+ * shared budget.  The CTAs of a (sequence, KV head) wait for one another at one
+ * point, with a bounded wait (DSA_ERR_DEVICE_TIMEOUT if it gives up).
  */
 int dsa_select(const void *q_blk, const void *k_cache, const void *v_cache,
                const int32_t *n_ctx, int32_t page, const int32_t *topk,
